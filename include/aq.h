@@ -1,0 +1,200 @@
+/*
+ * aq.h -- C ABI of libaq: tile-aligned mixed W4/W8 x A8 linear layers on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation is the linear projection Y = X W^T of the AlignQuant paper
+ * ("AlignQuant: Tile-Aligned Mixed-Precision Quantization for Efficient LLM
+ * Generation", arXiv 2610.07457; Sec. 3.1 defines the projection, Sec. 3.2
+ * and App. E.1/E.2 the packed representation, Sec. 3.3 and App. E.3 eq. 19
+ * the execution).  W (N x K) is cut into equal bN x bK tiles; every tile holds
+ * exactly one integer representation, INT4 or INT8, and one fp16 scale per
+ * output row.  X (M x K, bf16) is quantized per token to INT8.  The result is
+ *
+ *     y[m][n] = sx[m] * sum_j sw[n][j] * P[m][n][j]  (+ bias[n])
+ *     P[m][n][j] = sum_{k in tile column j} xq[m][k] * q[n][k]   (exact INT32)
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller unless a
+ *    comment says "host".  The library never frees caller memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Hot-path calls (aq_quant_act, aq_linear_decode, aq_linear_prefill) are
+ *    asynchronous on `stream`: they enqueue kernels and return; they neither
+ *    allocate nor synchronize, so they can be recorded into a CUDA graph.
+ *  - Arguments are validated on the host before any launch; a rejected call
+ *    launches nothing and returns a negative aq_status.  A launch failure
+ *    returns AQ_ERR_CUDA.  Errors found by a kernel while it runs (a bounded
+ *    wait that gave up) are recorded in the workspace and reported by
+ *    aq_workspace_status().
+ *  - Geometry: bN in {64, 128}, bK == 128, N % bN == 0, K % bK == 0.
+ *  - Row-major everywhere; leading dimensions are in elements.
+ */
+#ifndef AQ_H_
+#define AQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  AQ_OK = 0,
+  AQ_ERR_ARG = -1,         /* null pointer, bad enum, misaligned pointer, M/K/ld out of range */
+  AQ_ERR_SHAPE = -2,       /* N, K, bN, bK violate the tile geometry */
+  AQ_ERR_RANGE = -3,       /* an INT4 tile holds a code outside [-8, 7] (aq_pack) */
+  AQ_ERR_UNSUPPORTED = -4, /* a valid request this build does not implement */
+  AQ_ERR_WORKSPACE = -5,   /* workspace missing or smaller than aq_workspace_bytes() */
+  AQ_ERR_CUDA = -6,        /* a CUDA runtime call or a kernel launch failed */
+  AQ_ERR_TIMEOUT = -7      /* a kernel gave up on a bounded wait (see aq_workspace_status) */
+} aq_status;
+
+typedef enum { AQ_F32 = 0, AQ_BF16 = 1 } aq_dtype;
+typedef enum { AQ_PHASE_DECODE = 0, AQ_PHASE_PREFILL = 1 } aq_phase;
+
+/*
+ * One packed projection (App. E.1, E.2).  Every pointer is a device buffer
+ * owned by the caller and sized by aq_packed_sizes(); aq_pack() fills them.
+ *
+ *  bitmap   uint8  [ceil(R*C/8)]   precision label beta_{r,j} of logical tile
+ *                                  t = r*C + j is bit (t % 8) of byte t / 8
+ *                                  (row-major order, first label in the LSB);
+ *                                  beta = 1 marks an INT4 tile.
+ *  row_off4 int32  [R+1]           INT4 tiles in tile rows < r (eq. 16, first sum)
+ *  row_off8 int32  [R+1]           INT8 tiles in tile rows < r
+ *  tile_idx int32  [R*C]           physical index of logical tile t inside its
+ *                                  precision's buffer (eq. 16 evaluated once)
+ *  w4       uint8  [T4][bN][bK/2]  INT4 tiles in row order; byte i of a tile row
+ *                                  holds k = 2i in its low nibble and k = 2i+1 in
+ *                                  its high nibble (eq. 17), two's complement
+ *  w8       int8   [T8][bN][bK]    INT8 tiles in row order, row-major in the tile
+ *  scales   fp16   [R][C][bN]      sw[n][j] at (r*C + j)*bN + (n - r*bN), bits
+ *                                  as uint16, logical tile order
+ *
+ * Inside a tile both precisions use the same element order: output row, then
+ * input column.
+ */
+typedef struct aq_packed {
+  int32_t N, K, bN, bK, R, C, T4, T8;
+  uint8_t* bitmap;
+  int32_t* row_off4;
+  int32_t* row_off8;
+  int32_t* tile_idx;
+  uint8_t* w4;
+  int8_t* w8;
+  uint16_t* scales;
+} aq_packed;
+
+/* Index of each buffer in the size array of aq_packed_sizes(). */
+enum {
+  AQ_BUF_BITMAP = 0, AQ_BUF_ROW_OFF4 = 1, AQ_BUF_ROW_OFF8 = 2, AQ_BUF_TILE_IDX = 3,
+  AQ_BUF_W4 = 4, AQ_BUF_W8 = 5, AQ_BUF_SCALES = 6, AQ_NUM_BUFS = 7
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* aq_status_str(int status);
+
+/*
+ * Host only, no CUDA call.  Byte size of each of the seven packed buffers for
+ * an N x K projection with bN x bK tiles of which T4 are INT4.
+ * out_bytes: host array of AQ_NUM_BUFS entries.
+ * Errors: AQ_ERR_ARG (null out_bytes, T4 outside [0, R*C]), AQ_ERR_SHAPE.
+ */
+int aq_packed_sizes(int N, int K, int bN, int bK, int T4, size_t* out_bytes);
+
+/*
+ * Host only, no CUDA call.  Metadata of the packed format from a HOST copy of
+ * the precision labels map[R][C] (1 = INT4, 0 = INT8): bitmap, both row-offset
+ * arrays and tile_idx, written to HOST buffers of the sizes aq_packed_sizes()
+ * gives.  *T4_out (nullable) receives the INT4 tile count.
+ * Errors: AQ_ERR_ARG (null pointer, R or C < 1, a label other than 0 or 1).
+ * Follows App. E.1 and eq. 16.
+ */
+int aq_pack_metadata(const uint8_t* map_host, int R, int C, uint8_t* bitmap, int32_t* row_off4,
+                     int32_t* row_off8, int32_t* tile_idx, int32_t* T4_out);
+
+/*
+ * Pack integer codes into the tile format (App. E.1, E.2; eq. 16, 17).
+ *  codes  int8  [N][K] device, row-major: INT8 tiles any value, INT4 tiles in [-8, 7]
+ *  scales fp16  [N][C] device (bits as uint16), sw[n][j]
+ *  map    uint8 [R][C] device, 1 = INT4 tile, 0 = INT8 tile
+ *  out    host struct whose seven pointers the caller set to device buffers of
+ *         aq_packed_sizes(N, K, bN, bK, out->T4) bytes; out->T4 must equal the
+ *         number of INT4 labels in map.  The remaining fields are filled in.
+ * Offline step: synchronizes `stream` and allocates a few bytes of temporary
+ * device memory.  Errors: AQ_ERR_ARG (also when out->T4 disagrees with map),
+ * AQ_ERR_SHAPE, AQ_ERR_RANGE (an INT4 tile holds a code outside [-8, 7]; the
+ * output buffers are then unspecified), AQ_ERR_CUDA.
+ */
+int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_t* map, int N, int K, int bN,
+            int bK, aq_packed* out, void* stream);
+
+/*
+ * Per-token symmetric INT8 quantization of activations (App. B.3 computed per
+ * token; eq. 5 rounding; eq. 6 floor), in fp64:
+ *   s = max(max_k |x[m][k]| / 127, 1e-12);  xq[m][k] = clamp(rint(x[m][k] / s), -127, 127)
+ *   sx[m] = (float)s          (codes use the fp64 s; rint rounds half to even)
+ *  x   bf16 [M][ldx] device (bits as uint16), 16-byte aligned, ldx % 8 == 0, ldx >= K
+ *  xq  int8 [M][K] device, 16-byte aligned
+ *  sx  fp32 [M] device
+ * 1 <= M, 16 <= K <= 1048576 with K % 16 == 0.  Errors: AQ_ERR_ARG, AQ_ERR_CUDA.
+ */
+int aq_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream);
+
+/*
+ * Device scratch bytes a linear call needs for `phase` (aq_phase) at M tokens
+ * with packed weights *w (host struct; only its geometry is read).  Host only.
+ * The workspace must be zero-filled once when allocated; afterwards the library
+ * leaves it ready for the next call.  Calls that share a workspace must not run
+ * concurrently.  Returns 0 when the arguments are invalid.
+ */
+size_t aq_workspace_bytes(int phase, int M, const aq_packed* w);
+
+/*
+ * Decode-phase linear layer, 1 <= M <= 64 (Sec. 3.3 "Decode parallelism";
+ * App. E.3 eq. 19 and the ordered split reduction after it).
+ *  w     host struct describing device buffers produced by aq_pack
+ *  xq    int8 [M][K] device, 16-byte aligned (from aq_quant_act)
+ *  sx    fp32 [M] device
+ *  bias  fp32 [N] device or NULL
+ *  y     [M][ldy] device, fp32 or bf16 per ydtype (aq_dtype), ldy >= N
+ *  ws    device workspace of >= aq_workspace_bytes(AQ_PHASE_DECODE, M, w) bytes
+ * Split-K partial sums are reduced in increasing split order, so results are
+ * bitwise reproducible for a given (M, w) on a given GPU.
+ * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ */
+int aq_linear_decode(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                     void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Prefill-phase linear layer, any M >= 1 (Sec. 3.3 "Prefill weight reuse";
+ * App. E.3 eq. 19).  Same arguments as aq_linear_decode; the workspace size is
+ * aq_workspace_bytes(AQ_PHASE_PREFILL, M, w).  INT4 tiles are expanded to INT8
+ * on chip and the INT8 products run on the tensor cores (tcgen05).
+ * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ */
+int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                      void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Test entry: the exact per-tile INT32 products P[m][n][j] (eq. 19, the
+ * parenthesized product) written to P int32 [M][N][C] device, computed by the
+ * same data path (tile location, INT4 expansion, integer products) as the
+ * linear call of `phase`.  Not a hot-path call.
+ * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ */
+int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int M, int phase, int32_t* P,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the error word a kernel left in
+ * the workspace `ws`.  Returns AQ_OK, AQ_ERR_TIMEOUT (a bounded wait inside a
+ * kernel gave up; *info, nullable, receives where) or AQ_ERR_CUDA.
+ */
+int aq_workspace_status(void* ws, void* stream, int* info);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQ_H_ */

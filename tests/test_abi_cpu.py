@@ -1,0 +1,128 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+include/aq.h declares, and its host-only logic (buffer sizing, packed-format
+metadata, argument validation) agrees with the oracle."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from w8_a8_quantized_b200 import aq, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "aq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(aq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("aq_pack", "aq_quant_act", "aq_linear_decode", "aq_linear_prefill"):
+        assert required in names
+    assert set(names) == set(aq.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    L = aq.lib()
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = aq.lib()
+    for code in range(0, -8, -1):
+        assert L.aq_status_str(code).decode().startswith("AQ_")
+    assert L.aq_status_str(12345).decode() == "unknown aq_status"
+
+
+@pytest.mark.parametrize("N,K,bN,T4", [(256, 512, 128, 3), (192, 384, 64, 0), (128, 128, 128, 1), (5120, 17408, 128, 3000)])
+def test_packed_sizes_match_oracle(N, K, bN, T4):
+    sz = aq.aq_packed_sizes(N, K, bN, 128, T4)
+    R, C = N // bN, K // 128
+    g = dict(N=N, bN=bN, bK=128, R=R, C=C, T4=T4, T8=R * C - T4)
+    assert sum(sz.values()) == oracle.packed_bytes(g)
+    assert sz["w4"] == T4 * bN * 64 and sz["w8"] == (R * C - T4) * bN * 128
+    assert sz["bitmap"] == (R * C + 7) // 8 and sz["scales"] == 2 * N * C
+
+
+@pytest.mark.parametrize("args,status", [
+    ((100, 128, 128, 128, 0), -2), ((128, 100, 128, 128, 0), -2), ((128, 128, 32, 128, 0), -2),
+    ((128, 128, 128, 64, 0), -2), ((128, 128, 128, 128, 2), -1), ((128, 128, 128, 128, -1), -1)])
+def test_packed_sizes_rejects(args, status):
+    out = (ctypes.c_size_t * 7)()
+    assert aq.lib().aq_packed_sizes(*args, out) == status
+
+
+def _metadata(pmap):
+    R, C = pmap.shape
+    T = R * C
+    bitmap = np.zeros((T + 7) // 8, np.uint8)
+    off4 = np.zeros(R + 1, np.int32)
+    off8 = np.zeros(R + 1, np.int32)
+    idx = np.zeros(T, np.int32)
+    t4 = ctypes.c_int32(-1)
+    m = np.ascontiguousarray(pmap, dtype=np.uint8)
+    rc = aq.lib().aq_pack_metadata(m.ctypes.data, R, C, bitmap.ctypes.data, off4.ctypes.data, off8.ctypes.data,
+                                   idx.ctypes.data, ctypes.byref(t4))
+    return rc, bitmap, off4, off8, idx, t4.value
+
+
+@pytest.mark.parametrize("R,C,frac8,seed", [(1, 3, 0.34, 0), (3, 5, 0.5, 1), (8, 24, 0.25, 2), (40, 136, 0.3, 3),
+                                            (7, 9, 0.0, 4), (7, 9, 1.0, 5)])
+def test_pack_metadata_matches_oracle(R, C, frac8, seed):
+    pmap = synth.precision_map(R, C, frac8, (seed,))
+    rc, bitmap, off4, off8, idx, t4 = _metadata(pmap)
+    assert rc == 0
+    assert np.array_equal(bitmap, oracle.labels_to_bitmap(pmap))
+    assert np.array_equal(off4, oracle.row_offsets(pmap, 4))
+    assert np.array_equal(off8, oracle.row_offsets(pmap, 8))
+    assert t4 == int(pmap.sum())
+    for r in range(R):
+        for j in range(C):
+            assert idx[r * C + j] == oracle.physical_index(pmap, r, j, 4 if pmap[r, j] else 8)
+
+
+def test_pack_metadata_worked_example_and_rejects_bad_label():
+    rc, bitmap, off4, off8, idx, t4 = _metadata(np.array([[1, 0, 1]], np.uint8))
+    assert rc == 0 and list(idx) == [0, 0, 1] and t4 == 2 and list(bitmap) == [5]
+    rc, *_ = _metadata(np.array([[1, 2, 0]], np.uint8))
+    assert rc == -1
+
+
+def test_host_validation_rejects_before_any_launch():
+    L = aq.lib()
+    # activation quantization: bad M, K, ldx and alignment
+    assert L.aq_quant_act(16, 0, 128, 128, 16, 16, None) == -1
+    assert L.aq_quant_act(16, 1, 100, 128, 16, 16, None) == -1
+    assert L.aq_quant_act(16, 1, 128, 64, 16, 16, None) == -1
+    assert L.aq_quant_act(17, 1, 128, 128, 16, 16, None) == -1
+    assert L.aq_quant_act(None, 1, 128, 128, 16, 16, None) == -1
+    # linear calls: null struct, bad geometry, M out of range, bad dtype
+    assert L.aq_linear_decode(None, 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    s = aq.AqPackedStruct(N=100, K=128, bN=128, bK=128, R=0, C=1, T4=0, T8=0)
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -2
+    s = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
+                          bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 65, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, None, 16, 7, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 64, 16, 1 << 20, None) == -1
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, None, 0, None) == -5
+    assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, 16, 8, None) == -5
+    assert L.aq_workspace_bytes(0, 65, ctypes.byref(s)) == 0
+    assert L.aq_workspace_bytes(0, 1, ctypes.byref(s)) >= 256
+    assert L.aq_workspace_bytes(5, 1, ctypes.byref(s)) == 0
+    assert L.aq_debug_tile_partials(ctypes.byref(s), 16, 1, 3, 16, 16, 1 << 20, None) == -1
+
+
+def test_decode_workspace_grows_with_splits_and_tokens():
+    L = aq.lib()
+    s = aq.AqPackedStruct(N=1024, K=3072, bN=128, bK=128, R=8, C=24, T4=100, T8=92,
+                          bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    b1 = L.aq_workspace_bytes(0, 1, ctypes.byref(s))
+    b8 = L.aq_workspace_bytes(0, 8, ctypes.byref(s))
+    assert b8 > b1 > 256

@@ -1,0 +1,171 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer and byte results (packed buffers, activation codes and scales, per-tile
+INT32 products) must be bit-exact.  Floating-point outputs must meet the
+tolerance in aq_testutil.assert_output_close.  Sizes span several tiles with
+ragged token counts and, for 64-row tiles, an odd number of tile rows."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from aq_testutil import assert_output_close, dev_bf16, dev_projection, oracle_linear, packed_case
+from w8_a8_quantized_b200 import aq, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _no_kernel_errors():
+    yield
+    aq.check_all_workspaces()
+
+
+# ------------------------------------------------------------------ packer
+
+@pytest.mark.parametrize("N,K,bN,frac8,seed", [
+    (256, 384, 128, 0.5, 1), (192, 256, 64, 0.25, 2), (128, 128, 128, 1.0, 3), (128, 256, 128, 0.0, 4),
+    (640, 1280, 64, 0.5, 5), (1024, 3072, 128, 0.25, 6)])
+def test_pack_matches_oracle(N, K, bN, frac8, seed):
+    p = synth.projection_inputs(N, K, bN, 128, frac8, (seed,))
+    w = aq.aq_pack(*dev_projection(p), bN, 128)
+    ref = oracle.pack(p.codes, p.scales, p.pmap, bN, 128)
+    got = w.host_buffers()
+    assert (w.T4, w.T8, w.R, w.C) == (ref["T4"], ref["T8"], ref["R"], ref["C"])
+    for name in aq.BUF_NAMES:
+        want = np.ascontiguousarray(ref[name]).view(np.uint8).reshape(-1)
+        assert np.array_equal(got[name], want), name
+
+
+def test_pack_rejects_int4_code_out_of_range():
+    p = synth.projection_inputs(256, 256, 128, 128, 0.5, (9,))
+    r, j = map(int, np.argwhere(p.pmap == 1)[0])
+    for bad in (8, -9):
+        codes = p.codes.copy()
+        codes[r * 128 + 3, j * 128 + 77] = bad
+        with pytest.raises(aq.AqError) as e:
+            aq.aq_pack(*dev_projection(synth.SingleProjection(p.N, p.K, 128, 128, p.pmap, codes, p.scales)), 128, 128)
+        assert e.value.status == -3
+
+
+# ------------------------------------------------------------------ activation quantization
+
+@pytest.mark.parametrize("M,K,pad,outlier", [(1, 128, 0, 0.0), (3, 2048, 8, 0.0), (17, 3072, 0, 0.01),
+                                             (2, 17408, 0, 0.01), (2, 40960, 16, 0.0), (64, 640, 0, 0.01)])
+def test_quant_act_bit_exact(M, K, pad, outlier):
+    x = synth.activations(M, K + pad, (M, K, pad), outlier_frac=outlier)
+    x[0, : K // 2] = 0                       # partial zero row
+    if M > 2:
+        x[2, :K] = 0                         # all-zero row: scale floor
+    xd = dev_bf16(x)
+    xq, sx = aq.aq_quant_act(xd, K=K)
+    xq_ref, sx_ref = oracle.quant_act(x[:, :K])
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), sx_ref.view(np.uint32))
+
+
+def test_quant_act_ties_round_half_even():
+    x = np.array([[127.0, 2.5, -2.5, 3.5, 0.5, 1.5, -0.5, -127.0] * 2], np.float32)
+    xq, sx = aq.aq_quant_act(dev_bf16(synth.f32_to_bf16_bits(x)))
+    assert list(xq.cpu().numpy()[0][:8]) == [127, 2, -2, 4, 0, 2, 0, -127]
+    assert sx.item() == 1.0
+
+
+# ------------------------------------------------------------------ exact per-tile products
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 16, 17, 33, 64])
+@pytest.mark.parametrize("bN", [128, 64])
+def test_decode_tile_products_bit_exact(M, bN):
+    p, x, w, xq, sx = packed_case(bN * 5, 128 * 6, bN, 0.5, 100 + M, M)
+    P = aq.aq_debug_tile_partials(w, xq, aq.AQ_PHASE_DECODE)
+    assert np.array_equal(xq.cpu().numpy(), oracle.quant_act(x)[0])
+    ref = oracle.tile_partials(p.codes, oracle.quant_act(x)[0], 128)
+    assert np.array_equal(P.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("M", [1, 64, 100, 257, 300])
+@pytest.mark.parametrize("bN,frac8", [(128, 0.5), (64, 0.25), (128, 0.0), (128, 1.0)])
+def test_prefill_tile_products_bit_exact(M, bN, frac8):
+    p, x, w, xq, sx = packed_case(bN * 5, 128 * 7, bN, frac8, 200 + M, M)
+    P = aq.aq_debug_tile_partials(w, xq, aq.AQ_PHASE_PREFILL)
+    ref = oracle.tile_partials(p.codes, oracle.quant_act(x)[0], 128)
+    assert np.array_equal(P.cpu().numpy(), ref)
+
+
+# ------------------------------------------------------------------ outputs
+
+@pytest.mark.parametrize("M", [1, 2, 4, 7, 8, 12, 16, 32, 40, 64])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_decode_matches_oracle(M, out_dtype):
+    N, K = 640, 1536
+    p, x, w, xq, sx = packed_case(N, K, 128, 0.25, 300 + M, M, outlier=0.01)
+    bias = np.linspace(-2, 2, N).astype(np.float32)
+    y = aq.aq_linear_decode(w, xq, sx, bias=torch.from_numpy(bias).cuda(), out_dtype=out_dtype)
+    assert_output_close(y, oracle_linear(p, x, bias=bias))
+
+
+@pytest.mark.parametrize("M", [1, 3, 8, 33])
+def test_decode_64_row_tiles_and_strided_output(M):
+    N, K = 64 * 7, 128 * 9
+    p, x, w, xq, sx = packed_case(N, K, 64, 0.5, 400 + M, M)
+    out = torch.full((M, N + 32), 7.0, device="cuda")
+    aq.aq_linear_decode(w, xq, sx, out=out[:, :N])
+    assert_output_close(out[:, :N], oracle_linear(p, x))
+    assert (out[:, N:] == 7.0).all()
+
+
+@pytest.mark.parametrize("M", [1, 50, 128, 300, 700])
+@pytest.mark.parametrize("bN,frac8", [(128, 0.4), (64, 0.3)])
+def test_prefill_matches_oracle(M, bN, frac8):
+    N, K = bN * 9, 128 * 10
+    p, x, w, xq, sx = packed_case(N, K, bN, frac8, 500 + M, M, outlier=0.01)
+    bias = np.linspace(-1, 1, N).astype(np.float32)
+    y = aq.aq_linear_prefill(w, xq, sx, bias=torch.from_numpy(bias).cuda())
+    assert_output_close(y, oracle_linear(p, x, bias=bias))
+    yb = aq.aq_linear_prefill(w, xq, sx, out_dtype=torch.bfloat16)
+    assert_output_close(yb, oracle_linear(p, x))
+
+
+def test_split_reduction_is_deterministic():
+    p, x, w, xq, sx = packed_case(1024, 3072, 128, 0.25, 600, 8)
+    ys = [aq.aq_linear_decode(w, xq, sx).cpu().numpy() for _ in range(3)]
+    assert all(np.array_equal(ys[0].view(np.uint32), y.view(np.uint32)) for y in ys[1:])
+    p, x, w, xq, sx = packed_case(1024, 3072, 128, 0.25, 601, 40)
+    ys = [aq.aq_linear_decode(w, xq, sx).cpu().numpy() for _ in range(3)]
+    assert all(np.array_equal(ys[0].view(np.uint32), y.view(np.uint32)) for y in ys[1:])
+
+
+@pytest.mark.parametrize("phase,M", [(0, 1), (0, 8), (0, 32), (1, 300)])
+def test_exact_sign_and_power_of_two_symmetry(phase, M):
+    """y(-X) = -y(X) and y(2^e X) = 2^e y(X) hold exactly for the GPU path too."""
+    p = synth.projection_inputs(512, 1024, 128, 128, 0.5, (700 + M,))
+    w = aq.aq_pack(*dev_projection(p), 128, 128)
+    x = synth.activations(M, 1024, (701 + M,))
+    xf = oracle.bf16_bits_to_f64(x).astype(np.float32)
+    run = aq.aq_linear_decode if phase == 0 else aq.aq_linear_prefill
+
+    def y_of(xbits):
+        xq, sx = aq.aq_quant_act(dev_bf16(xbits))
+        return run(w, xq, sx).cpu().numpy()
+
+    y = y_of(x)
+    assert np.array_equal(y_of(synth.f32_to_bf16_bits(-xf)), -y)
+    assert np.array_equal(y_of(synth.f32_to_bf16_bits(xf * np.float32(8.0))), y * 8)
+
+
+def test_decode_and_prefill_agree_on_products():
+    p, x, w, xq, sx = packed_case(384, 1024, 128, 0.5, 800, 24)
+    Pd = aq.aq_debug_tile_partials(w, xq, aq.AQ_PHASE_DECODE)
+    Pp = aq.aq_debug_tile_partials(w, xq, aq.AQ_PHASE_PREFILL)
+    assert torch.equal(Pd, Pp)
+
+
+def test_device_errors_are_reported():
+    p, x, w, xq, sx = packed_case(256, 256, 128, 0.5, 900, 4)
+    with pytest.raises(aq.AqError) as e:
+        aq.aq_linear_decode(w, xq, sx, ws=torch.zeros(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == -5
+    big = torch.zeros((65, 256), dtype=torch.int8, device="cuda")
+    with pytest.raises(aq.AqError) as e:
+        aq.aq_linear_decode(w, big, torch.ones(65, device="cuda"), ws=aq.workspace(0, 4, w))
+    assert e.value.status == -1

@@ -1,0 +1,240 @@
+"""Thin Python binding of libaq's C ABI (include/aq.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libaq.so.  PyTorch provides device memory and the current CUDA
+stream.  There is no CPU fallback: if libaq.so is missing the first call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libaq.so")
+
+AQ_OK = 0
+AQ_F32, AQ_BF16 = 0, 1
+AQ_PHASE_DECODE, AQ_PHASE_PREFILL = 0, 1
+BUF_NAMES = ("bitmap", "row_off4", "row_off8", "tile_idx", "w4", "w8", "scales")
+EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "aq_quant_act",
+            "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
+            "aq_workspace_status")
+
+
+class AqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().aq_status_str(status).decode()} ({status})")
+
+
+class AqPackedStruct(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("N", "K", "bN", "bK", "R", "C", "T4", "T8")] + \
+               [(n, ctypes.c_void_p) for n in BUF_NAMES]
+
+
+_lib = None
+
+
+def lib():
+    """Load libaq.so once and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m w8_a8_quantized_b200.build` "
+                           "(this package has no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    c_int, c_void_p, c_size_t = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+    P = ctypes.POINTER(AqPackedStruct)
+    L.aq_status_str.restype = ctypes.c_char_p
+    L.aq_status_str.argtypes = [c_int]
+    L.aq_packed_sizes.restype = c_int
+    L.aq_packed_sizes.argtypes = [c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_size_t)]
+    L.aq_pack_metadata.restype = c_int
+    L.aq_pack_metadata.argtypes = [c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   ctypes.POINTER(ctypes.c_int32)]
+    L.aq_pack.restype = c_int
+    L.aq_pack.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, P, c_void_p]
+    L.aq_quant_act.restype = c_int
+    L.aq_quant_act.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
+    L.aq_workspace_bytes.restype = c_size_t
+    L.aq_workspace_bytes.argtypes = [c_int, c_int, P]
+    for f in (L.aq_linear_decode, L.aq_linear_prefill):
+        f.restype = c_int
+        f.argtypes = [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p, c_size_t,
+                      c_void_p]
+    L.aq_debug_tile_partials.restype = c_int
+    L.aq_debug_tile_partials.argtypes = [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t, c_void_p]
+    L.aq_workspace_status.restype = c_int
+    L.aq_workspace_status.argtypes = [c_void_p, c_void_p, ctypes.POINTER(c_int)]
+    _lib = L
+    return L
+
+
+def _check(rc: int, what: str):
+    if rc != AQ_OK:
+        raise AqError(rc, what)
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype, device=None):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise TypeError(f"{name} must be a {dtype} tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def aq_packed_sizes(N: int, K: int, bN: int, bK: int, T4: int) -> dict:
+    out = (ctypes.c_size_t * 7)()
+    _check(lib().aq_packed_sizes(N, K, bN, bK, T4, out), "aq_packed_sizes")
+    return dict(zip(BUF_NAMES, [int(v) for v in out]))
+
+
+class PackedWeights:
+    """Device buffers of one packed projection plus the C struct describing them."""
+
+    def __init__(self, N: int, K: int, bN: int, bK: int, T4: int, device):
+        sizes = aq_packed_sizes(N, K, bN, bK, T4)
+        self.device = torch.device(device)
+        self.buffers = {n: torch.empty(max(s, 16), dtype=torch.uint8, device=self.device) for n, s in sizes.items()}
+        self.sizes = sizes
+        self.struct = AqPackedStruct(N=N, K=K, bN=bN, bK=bK, R=N // bN, C=K // bK, T4=T4, T8=0)
+        for n in BUF_NAMES:
+            setattr(self.struct, n, self.buffers[n].data_ptr())
+
+    N = property(lambda s: s.struct.N)
+    K = property(lambda s: s.struct.K)
+    bN = property(lambda s: s.struct.bN)
+    bK = property(lambda s: s.struct.bK)
+    R = property(lambda s: s.struct.R)
+    C = property(lambda s: s.struct.C)
+    T4 = property(lambda s: s.struct.T4)
+    T8 = property(lambda s: s.struct.T8)
+
+    @property
+    def nbytes(self) -> int:
+        """Bytes of the packed representation (all seven buffers)."""
+        return sum(self.sizes.values())
+
+    def host_buffers(self) -> dict:
+        return {n: self.buffers[n][: self.sizes[n]].cpu().numpy() for n in BUF_NAMES}
+
+
+def aq_pack(codes: torch.Tensor, scales: torch.Tensor, pmap: torch.Tensor, bN: int, bK: int) -> PackedWeights:
+    """codes int8 [N][K], scales float16 [N][C], pmap uint8 [R][C] (1 = INT4), all on one CUDA device."""
+    _need(codes, "codes", torch.int8)
+    dev = codes.device
+    _need(scales, "scales", torch.float16, dev)
+    _need(pmap, "pmap", torch.uint8, dev)
+    N, K = codes.shape
+    T4 = int(pmap.sum().item())
+    w = PackedWeights(N, K, bN, bK, T4, dev)
+    _check(lib().aq_pack(codes.data_ptr(), scales.data_ptr(), pmap.data_ptr(), N, K, bN, bK,
+                         ctypes.byref(w.struct), _stream(dev)), "aq_pack")
+    return w
+
+
+def aq_quant_act(x: torch.Tensor, xq: torch.Tensor = None, sx: torch.Tensor = None, K: int = None):
+    """x bf16 [M][ldx] -> (xq int8 [M][K], sx float32 [M]) on x's stream."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor with unit inner stride")
+    M = x.shape[0]
+    K = x.shape[1] if K is None else K
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if sx is None:
+        sx = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need(xq, "xq", torch.int8, x.device)
+    _need(sx, "sx", torch.float32, x.device)
+    _check(lib().aq_quant_act(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), sx.data_ptr(), _stream(x.device)),
+           "aq_quant_act")
+    return xq, sx
+
+
+def aq_workspace_bytes(phase: int, M: int, w: PackedWeights) -> int:
+    return int(lib().aq_workspace_bytes(phase, M, ctypes.byref(w.struct)))
+
+
+_ws_cache = {}
+
+
+def workspace(phase: int, M: int, w: PackedWeights) -> torch.Tensor:
+    """A zero-initialised workspace big enough for (phase, M, w), cached per device."""
+    need = aq_workspace_bytes(phase, M, w)
+    if need == 0:
+        raise ValueError("invalid arguments for a workspace")
+    key = (w.device, phase)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=w.device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _linear(fn, name, phase, w, xq, sx, bias, out, out_dtype, ws):
+    _need(xq, "xq", torch.int8, w.device)
+    _need(sx, "sx", torch.float32, w.device)
+    M = xq.shape[0]
+    if out is None:
+        out = torch.empty((M, w.N), dtype=out_dtype, device=w.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or out.stride(1) != 1 or out.device != w.device:
+        raise ValueError("out must be float32 or bfloat16 on the weights' device with unit inner stride")
+    ydt = AQ_F32 if out.dtype == torch.float32 else AQ_BF16
+    if bias is not None:
+        _need(bias, "bias", torch.float32, w.device)
+    if ws is None:
+        ws = workspace(phase, M, w)
+    _check(fn(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
+              bias.data_ptr() if bias is not None else None, out.data_ptr(), ydt, out.stride(0),
+              ws.data_ptr(), ws.numel(), _stream(w.device)), name)
+    return out
+
+
+def aq_linear_decode(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=torch.float32, ws=None):
+    """Decode-phase y = sx * sum_j sw * (xq q^T)_j (+ bias) for 1 <= M <= 64 tokens."""
+    return _linear(lib().aq_linear_decode, "aq_linear_decode", AQ_PHASE_DECODE, w, xq, sx, bias, out, out_dtype, ws)
+
+
+def aq_linear_prefill(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=torch.float32, ws=None):
+    """Prefill-phase y (tensor-core INT8 path), any M >= 1."""
+    return _linear(lib().aq_linear_prefill, "aq_linear_prefill", AQ_PHASE_PREFILL, w, xq, sx, bias, out, out_dtype,
+                   ws)
+
+
+def aq_debug_tile_partials(w: PackedWeights, xq: torch.Tensor, phase: int, ws=None) -> torch.Tensor:
+    """Exact INT32 tile products P[M][N][C] computed by the `phase` data path."""
+    _need(xq, "xq", torch.int8, w.device)
+    M = xq.shape[0]
+    P = torch.zeros((M, w.N, w.C), dtype=torch.int32, device=w.device)
+    if ws is None:
+        ws = workspace(AQ_PHASE_PREFILL, M, w)
+    _check(lib().aq_debug_tile_partials(ctypes.byref(w.struct), xq.data_ptr(), M, phase, P.data_ptr(),
+                                        ws.data_ptr(), ws.numel(), _stream(w.device)), "aq_debug_tile_partials")
+    return P
+
+
+def aq_workspace_status(ws: torch.Tensor):
+    """Synchronise; return (status, info) of the kernel error word of a workspace and clear it."""
+    info = ctypes.c_int(0)
+    rc = lib().aq_workspace_status(ws.data_ptr(), _stream(ws.device), ctypes.byref(info))
+    if rc not in (AQ_OK, -7):
+        _check(rc, "aq_workspace_status")
+    return rc, info.value
+
+
+def check_all_workspaces():
+    """Raise if any cached workspace recorded a kernel error."""
+    for ws in _ws_cache.values():
+        rc, info = aq_workspace_status(ws)
+        if rc != AQ_OK:
+            raise AqError(rc, f"kernel wait gave up (info {info})")

@@ -1,0 +1,163 @@
+// C ABI entry points of libaq: host-side validation, split planning and
+// dispatch to the sm_100a kernels.  Every hot-path entry validates its
+// arguments, enqueues its kernels on the caller's stream and returns without
+// allocating or synchronizing.
+#include <algorithm>
+
+#include "aq_internal.cuh"
+
+namespace aq {
+
+int validate_packed(const aq_packed* w) {
+  if (!w) return AQ_ERR_ARG;
+  if (!geometry_ok(w->N, w->K, w->bN, w->bK)) return AQ_ERR_SHAPE;
+  if (w->R != w->N / w->bN || w->C != w->K / w->bK) return AQ_ERR_SHAPE;
+  if (w->T4 < 0 || w->T8 < 0 || (long long)w->T4 + w->T8 != (long long)w->R * w->C) return AQ_ERR_SHAPE;
+  if (!w->bitmap || !w->row_off4 || !w->row_off8 || !w->tile_idx || !w->scales) return AQ_ERR_ARG;
+  if ((w->T4 > 0 && !w->w4) || (w->T8 > 0 && !w->w8)) return AQ_ERR_ARG;
+  if (((uintptr_t)w->w4 & 15) || ((uintptr_t)w->w8 & 15)) return AQ_ERR_ARG;
+  return AQ_OK;
+}
+
+static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, dp4a has room);
+// more tokens on the tensor cores.  Splits over tile columns fill the GPU.
+DecodePlan plan_decode(int M, const aq_packed* w) {
+  DecodePlan p;
+  if (M <= 8) {
+    p.kernel = 0;
+    p.rows = w->bN;
+    p.blocks = w->R;
+    p.S = std::max(1, std::min(w->C, ceil_div(2 * kNumSMs, p.blocks)));
+  } else {
+    p.kernel = 1;
+    p.rows = 128;
+    p.blocks = ceil_div(w->R, 128 / w->bN);
+    p.S = std::max(1, std::min(w->C, ceil_div(kNumSMs, p.blocks)));
+  }
+  return p;
+}
+
+static size_t counters_bytes(int blocks) { return ((size_t)blocks * sizeof(int) + 255) / 256 * 256; }
+
+size_t decode_ws_bytes(int M, const aq_packed* w) {
+  const DecodePlan p = plan_decode(M, w);
+  size_t b = kWsHeader + counters_bytes(p.blocks);
+  if (p.S > 1) b += (size_t)p.S * M * w->N * sizeof(float);
+  return b;
+}
+
+size_t prefill_ws_bytes(int /*M*/, const aq_packed* w) { return kWsHeader + counters_bytes(w->R); }
+
+}  // namespace aq
+
+using namespace aq;
+
+extern "C" const char* aq_status_str(int status) {
+  switch (status) {
+    case AQ_OK: return "AQ_OK";
+    case AQ_ERR_ARG: return "AQ_ERR_ARG: invalid argument";
+    case AQ_ERR_SHAPE: return "AQ_ERR_SHAPE: shape violates the tile geometry";
+    case AQ_ERR_RANGE: return "AQ_ERR_RANGE: INT4 tile holds a code outside [-8, 7]";
+    case AQ_ERR_UNSUPPORTED: return "AQ_ERR_UNSUPPORTED: not implemented by this build";
+    case AQ_ERR_WORKSPACE: return "AQ_ERR_WORKSPACE: workspace missing or too small";
+    case AQ_ERR_CUDA: return "AQ_ERR_CUDA: CUDA runtime or launch failure";
+    case AQ_ERR_TIMEOUT: return "AQ_ERR_TIMEOUT: a kernel gave up on a bounded wait";
+    default: return "unknown aq_status";
+  }
+}
+
+extern "C" int aq_packed_sizes(int N, int K, int bN, int bK, int T4, size_t* out) {
+  if (!out) return AQ_ERR_ARG;
+  if (!geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
+  const long long R = N / bN, C = K / bK, T = R * C;
+  if (T4 < 0 || T4 > T) return AQ_ERR_ARG;
+  const long long B = (long long)bN * bK;
+  out[AQ_BUF_BITMAP] = (size_t)((T + 7) / 8);
+  out[AQ_BUF_ROW_OFF4] = (size_t)(4 * (R + 1));
+  out[AQ_BUF_ROW_OFF8] = (size_t)(4 * (R + 1));
+  out[AQ_BUF_TILE_IDX] = (size_t)(4 * T);
+  out[AQ_BUF_W4] = (size_t)(B / 2 * T4);
+  out[AQ_BUF_W8] = (size_t)(B * (T - T4));
+  out[AQ_BUF_SCALES] = (size_t)(2 * T * bN);
+  return AQ_OK;
+}
+
+extern "C" size_t aq_workspace_bytes(int phase, int M, const aq_packed* w) {
+  if (validate_packed(w) != AQ_OK || M < 1) return 0;
+  if (phase == AQ_PHASE_DECODE) return M <= kMaxDecodeM ? decode_ws_bytes(M, w) : 0;
+  if (phase == AQ_PHASE_PREFILL) return prefill_ws_bytes(M, w);
+  return 0;
+}
+
+extern "C" int aq_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream) {
+  if (!x || !xq || !sx || M < 1 || K < 16 || K % 16 || K > (1 << 20) || ldx < K || ldx % 8) return AQ_ERR_ARG;
+  if (((uintptr_t)x & 15) || ((uintptr_t)xq & 15)) return AQ_ERR_ARG;
+  return launch_quant_act(x, M, K, ldx, xq, sx, static_cast<cudaStream_t>(stream)) == cudaSuccess ? AQ_OK
+                                                                                                   : AQ_ERR_CUDA;
+}
+
+static int check_linear(const aq_packed* w, const int8_t* xq, const float* sx, int M, const void* y, int ydtype,
+                        int ldy) {
+  int rc = validate_packed(w);
+  if (rc != AQ_OK) return rc;
+  if (!xq || !sx || !y || M < 1 || ldy < w->N) return AQ_ERR_ARG;
+  if (ydtype != AQ_F32 && ydtype != AQ_BF16) return AQ_ERR_ARG;
+  if ((uintptr_t)xq & 15) return AQ_ERR_ARG;
+  return AQ_OK;
+}
+
+extern "C" int aq_linear_decode(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                                void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_linear(w, xq, sx, M, y, ydtype, ldy);
+  if (rc != AQ_OK) return rc;
+  if (M > kMaxDecodeM) return AQ_ERR_ARG;
+  if (!ws || ws_bytes < decode_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const DecodePlan p = plan_decode(M, w);
+  cudaError_t e = p.kernel == 0 ? launch_decode_simt(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, st)
+                                : launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_DECODE, st);
+  return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+}
+
+extern "C" int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                                 void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_linear(w, xq, sx, M, y, ydtype, ldy);
+  if (rc != AQ_OK) return rc;
+  if (!ws || ws_bytes < prefill_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
+  cudaError_t e = launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_PREFILL,
+                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+}
+
+extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int M, int phase, int32_t* P, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  int rc = validate_packed(w);
+  if (rc != AQ_OK) return rc;
+  if (!xq || !P || M < 1 || ((uintptr_t)xq & 15)) return AQ_ERR_ARG;
+  if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return AQ_ERR_ARG;
+  if (phase == AQ_PHASE_DECODE && M > kMaxDecodeM) return AQ_ERR_ARG;
+  if (!ws || ws_bytes < kWsHeader) return AQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (phase == AQ_PHASE_DECODE && plan_decode(M, w).kernel == 0)
+    e = launch_decode_simt(w, xq, nullptr, M, nullptr, nullptr, AQ_F32, w->N, ws, P, st);
+  else
+    e = launch_tc(w, xq, nullptr, M, nullptr, nullptr, AQ_F32, w->N, ws, P, phase, st);
+  return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+}
+
+extern "C" int aq_workspace_status(void* ws, void* stream, int* info) {
+  if (!ws) return AQ_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  WsHeader h{0, 0};
+  if (cudaStreamSynchronize(st) != cudaSuccess) return AQ_ERR_CUDA;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return AQ_ERR_CUDA;
+  if (h.err_code != 0) {
+    const WsHeader zero{0, 0};
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return AQ_ERR_CUDA;
+  }
+  if (info) *info = h.err_info;
+  return h.err_code == 0 ? AQ_OK : AQ_ERR_TIMEOUT;
+}

@@ -71,11 +71,11 @@ def weight_codes(N: int, K: int, pmap: np.ndarray, bN: int, bK: int, seed) -> np
     """int8[N][K]: uniform over the full INT8 range, or over [-8, 7] in INT4 tiles."""
     R, C = pmap.shape
     assert R * bN == N and C * bK == K
-    raw = np.frombuffer(_rng(*_key(seed), 2).bytes(N * K), dtype=np.uint8).reshape(R, bN, C, bK)
-    as_int8 = raw.view(np.int8)
-    as_int4 = ((raw & 15).astype(np.int16) - 8).astype(np.int8)
-    is4 = pmap.astype(bool)[:, None, :, None]
-    return np.where(is4, as_int4, as_int8).reshape(N, K)
+    words = np.random.PCG64(np.random.SeedSequence(list(_key(seed)) + [2])).random_raw((N * K + 7) // 8)
+    raw = words.view(np.uint8)[: N * K].reshape(R, bN, C, bK)
+    # INT4 tiles: (b & 15) - 8, computed modulo 256 as (b & 15) + 248
+    np.copyto(raw, (raw & np.uint8(15)) + np.uint8(248), where=pmap.astype(bool)[:, None, :, None])
+    return raw.view(np.int8).reshape(N, K)
 
 
 def weight_scales(N: int, C: int, seed) -> np.ndarray:
