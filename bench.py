@@ -68,6 +68,8 @@ def parse():
     ap.add_argument("--workload", default="decode-llama-3.2-3b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None, help="measure only this token count")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     return ap.parse_args()
 
 
@@ -191,26 +193,45 @@ class Model:
         self.xq = {k: torch.empty((M, K), dtype=torch.int8, device=self.dev) for k, K in self.in_dims.items()}
         self.sx = {k: torch.empty((M,), dtype=torch.float32, device=self.dev) for k in self.in_dims}
         self.y = {n: torch.empty((M, N), dtype=torch.float32, device=self.dev) for n, N in self.out_dims.items()}
-        phase = aq.AQ_PHASE_DECODE if self.wl["phase"] == "decode" else aq.AQ_PHASE_PREFILL
-        need = max(aq.aq_workspace_bytes(phase, M, w) for layer in self.weights for w in layer.values())
+        self.phase = aq.AQ_PHASE_DECODE if self.wl["phase"] == "decode" else aq.AQ_PHASE_PREFILL
+        self.members = {}
+        for name, _, _ in self.projs:
+            self.members.setdefault(INPUT_OF[name], []).append(name)
+        self.groups = [{kind: aq.Group([self.weights[l][n] for n in names], self.phase, M)
+                        for kind, names in self.members.items()} for l in range(self.layers)]
+        need = max([g.ws.numel() for layer in self.groups for g in layer.values()] +
+                   [aq.aq_workspace_bytes(self.phase, M, w) for layer in self.weights for w in layer.values()])
+        for layer in self.groups:
+            for g in layer.values():
+                g.ws = None  # one shared workspace (the step runs in stream order)
         self.ws = torch.zeros(need, dtype=torch.uint8, device=self.dev)
-        self.run = aq.aq_linear_decode if phase == aq.AQ_PHASE_DECODE else aq.aq_linear_prefill
+        self.run = aq.aq_linear_decode if self.phase == aq.AQ_PHASE_DECODE else aq.aq_linear_prefill
+        # input kinds whose group runs as one fused launch (activation preparation inside)
+        self.fused = self.phase == aq.AQ_PHASE_DECODE and M <= 8
 
-    def step(self, linears=True, quant=True):
-        """Enqueue one pass; returns the number of kernel launches."""
+    def step(self, mode="group"):
+        """Enqueue one pass; returns the number of kernel launches.
+
+        mode "group": the hot path, one aq_linear_group call per shared input
+        (query/key/value, attention output, gate/up, MLP hidden) per layer.
+        mode "linear": only the linear kernels on already-quantized inputs."""
         aq = self.aq
         n = 0
         for l in range(self.layers):
-            for kind in self.in_dims:
-                if quant:
-                    aq.aq_quant_act(self.x[l][kind], self.xq[kind], self.sx[kind])
-                    n += 1
-            if linears:
-                for name, _, _ in self.projs:
-                    kind = INPUT_OF[name]
-                    self.run(self.weights[l][name], self.xq[kind], self.sx[kind], out=self.y[name], ws=self.ws)
-                    n += 1
+            for kind, names in self.members.items():
+                if mode == "group":
+                    self.groups[l][kind](self.x[l][kind], [self.y[nm] for nm in names], ws=self.ws)
+                    n += 1 if self.fused else 1 + len(names)  # fused launch, or quantize + members
+                else:
+                    for nm in names:
+                        self.run(self.weights[l][nm], self.xq[kind], self.sx[kind], out=self.y[nm], ws=self.ws)
+                        n += 1
         return n
+
+    def quantize_inputs(self):
+        """Fill the pre-quantized inputs used by mode "linear" (from layer 0's activations)."""
+        for kind in self.members:
+            self.aq.aq_quant_act(self.x[0][kind], self.xq[kind], self.sx[kind])
 
     def graph(self, **kw):
         torch = self.torch
@@ -233,10 +254,12 @@ def time_graph(torch, g, steps, warmup, dist_on, dev):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("aq_timed")
     e0.record()
     for _ in range(steps):
         g.replay()
     e1.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(dev)
     if dist_on:
         torch.distributed.barrier()
@@ -347,29 +370,36 @@ def main():
     from w8_a8_quantized_b200 import aq
     aq.lib()
 
+    Ms = [wl["M"], *wl["extra_M"]] if args.tokens is None else [args.tokens]
     t_setup = time.time()
-    model = Model(wl, wl["M"], dev, rank)
+    model = Model(wl, Ms[0], dev, rank)
     setup_s = time.time() - t_setup
 
     results = {}
-    Ms = [wl["M"], *wl["extra_M"]]
     clocks = None
     for M in Ms:
         if M != model.M:
             model.set_tokens(M)
         g, launches = model.graph()
-        if M == wl["M"]:
+        if M == Ms[0]:
             with ClockSampler(local) as cs:
                 ms = time_graph(torch, g, args.steps, args.warmup, dist_on, dev)
             clocks = cs.summary()
         else:
             ms = time_graph(torch, g, args.steps, args.warmup, dist_on, dev)
-        g_lin, lin_launches = model.graph(quant=False)
-        ms_lin = time_graph(torch, g_lin, args.steps, args.warmup, dist_on, dev)
+        if model.fused:  # the step holds nothing but the dominant (fused decode) kernel
+            g_lin, lin_launches, ms_lin = None, launches, ms
+        else:
+            model.quantize_inputs()
+            g_lin, lin_launches = model.graph(mode="linear")
+            ms_lin = time_graph(torch, g_lin, args.steps, args.warmup, dist_on, dev)
         res = dict(ms=ms, launches=launches, ms_linear_only=ms_lin, linear_launches=lin_launches)
-        if M == wl["M"]:
-            ms_e2e, h2d, d2h = time_e2e(torch, model, g, args.steps, args.warmup, dev)
-            res.update(ms_e2e=ms_e2e, h2d=h2d, d2h=d2h)
+        if M == Ms[0]:
+            if args.no_e2e:
+                res.update(ms_e2e=float("nan"), h2d=0, d2h=0)
+            else:
+                ms_e2e, h2d, d2h = time_e2e(torch, model, g, args.steps, args.warmup, dev)
+                res.update(ms_e2e=ms_e2e, h2d=h2d, d2h=d2h)
         results[M] = res
         aq.check_all_workspaces()
         rc, info = aq.aq_workspace_status(model.ws)
@@ -377,7 +407,7 @@ def main():
             raise RuntimeError(f"kernel reported error {rc} ({info})")
         del g, g_lin
 
-    r0 = results[wl["M"]]
+    r0 = results[Ms[0]]
     decode = wl["phase"] == "decode"
     wbytes = model.weight_bytes
     if decode:
@@ -405,7 +435,7 @@ def main():
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r0["ms"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded random codes, scales, maps, activations)",
-        "config": {"workload": args.workload, "model_shape": wl["model"], "phase": wl["phase"], "tokens": wl["M"],
+        "config": {"workload": args.workload, "model_shape": wl["model"], "phase": wl["phase"], "tokens": Ms[0],
                    "tile": [wl["bN"], 128], "int8_tile_fraction": wl["frac8"], "layers": model.layers,
                    "projections_per_layer": 7, "packed_weight_bytes": wbytes, "parallelism": f"replicas x{world}",
                    "l2": "not flushed: weights streamed per step exceed the 126 MB L2", "graph": "one CUDA graph per step"},
@@ -431,7 +461,8 @@ def main():
         pm = Model(pwl, pwl["M"], dev, rank)
         g, launches = pm.graph()
         ms = time_graph(torch, g, max(3, args.steps // 2), max(3, args.warmup), dist_on, dev)
-        g_lin, _ = pm.graph(quant=False)
+        pm.quantize_inputs()
+        g_lin, _ = pm.graph(mode="linear")
         ms_lin = time_graph(torch, g_lin, max(3, args.steps // 2), max(3, args.warmup), dist_on, dev)
         ops = 2.0 * pm.M * pm.macs
         int8_peak = 2.0 * peaks["bf16"]

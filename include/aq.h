@@ -187,6 +187,33 @@ int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int M, int phas
                            void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Shared-input projection group (Sec. 3.3 "Shared activation preparation";
+ * App. E.4): G (1..3) projections that read the same activations, e.g. query /
+ * key / value or gate / up, prepared once and computed in as few launches as
+ * possible.  For every member g:  y[g] = linear(w[g], quant(x)) (+ bias[g]),
+ * exactly as aq_quant_act followed by aq_linear_decode / aq_linear_prefill.
+ *  phase  AQ_PHASE_DECODE (1 <= M <= 64) or AQ_PHASE_PREFILL (M >= 1)
+ *  w      host array of G pointers to packed projections with equal K
+ *  x      bf16 [M][ldx] device (bits as uint16), 16-byte aligned, ldx % 8 == 0
+ *  bias   host array of G device pointers (each fp32 [N_g] or NULL), or NULL
+ *  y      host array of G device outputs [M][ldy[g]], fp32 or bf16 per ydtype
+ *  ldy    host array of G leading dimensions, ldy[g] >= N_g
+ *  ws     device workspace of >= aq_group_workspace_bytes(phase, M, w, G) bytes
+ * Decode with at most 8 tokens runs as ONE launch: every CTA quantizes the
+ * input it needs itself (same arithmetic as aq_quant_act) and the members'
+ * output rows are concatenated.  Other cases quantize x once into the
+ * workspace and run each member on it.
+ * Errors: AQ_ERR_ARG (also G outside 1..3, unequal K), AQ_ERR_SHAPE,
+ * AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ */
+int aq_linear_group(int phase, const aq_packed* const* w, int G, const uint16_t* x, int ldx, int M,
+                    const float* const* bias, void* const* y, const int* ldy, int ydtype, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Host only.  Workspace bytes of aq_linear_group(phase, ..., M, w, G); 0 when invalid. */
+size_t aq_group_workspace_bytes(int phase, int M, const aq_packed* const* w, int G);
+
+/*
  * Synchronizes `stream`, then reads and clears the error word a kernel left in
  * the workspace `ws`.  Returns AQ_OK, AQ_ERR_TIMEOUT (a bounded wait inside a
  * kernel gave up; *info, nullable, receives where) or AQ_ERR_CUDA.

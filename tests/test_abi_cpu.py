@@ -119,10 +119,33 @@ def test_host_validation_rejects_before_any_launch():
     assert L.aq_debug_tile_partials(ctypes.byref(s), 16, 1, 3, 16, 16, 1 << 20, None) == -1
 
 
-def test_decode_workspace_grows_with_splits_and_tokens():
+def test_decode_workspace_sizes():
+    """Up to 8 tokens the CUDA-core kernel needs only the status header; above,
+    the tensor-core split-K partial sums grow with the token count."""
     L = aq.lib()
     s = aq.AqPackedStruct(N=1024, K=3072, bN=128, bK=128, R=8, C=24, T4=100, T8=92,
                           bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
     b1 = L.aq_workspace_bytes(0, 1, ctypes.byref(s))
     b8 = L.aq_workspace_bytes(0, 8, ctypes.byref(s))
-    assert b8 > b1 > 256
+    b16 = L.aq_workspace_bytes(0, 16, ctypes.byref(s))
+    b32 = L.aq_workspace_bytes(0, 32, ctypes.byref(s))
+    assert b1 == b8 == 256
+    assert b32 > b16 > 256
+
+
+def test_group_workspace_sizes():
+    L = aq.lib()
+    P = ctypes.POINTER(aq.AqPackedStruct)
+    mk = lambda N: aq.AqPackedStruct(N=N, K=3072, bN=128, bK=128, R=N // 128, C=24, T4=0, T8=(N // 128) * 24,
+                                     bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    q, k, v = mk(3072), mk(1024), mk(1024)
+    arr = (P * 3)(ctypes.pointer(q), ctypes.pointer(k), ctypes.pointer(v))
+    assert L.aq_group_workspace_bytes(0, 1, arr, 3) == 256          # fused: one launch, no scratch
+    assert L.aq_group_workspace_bytes(0, 16, arr, 3) >= 16 * 3072   # quantized input kept in the workspace
+    assert L.aq_group_workspace_bytes(1, 300, arr, 3) >= 300 * 3072
+    assert L.aq_group_workspace_bytes(0, 65, arr, 3) == 0
+    assert L.aq_group_workspace_bytes(0, 1, arr, 4) == 0
+    bad = mk(1024)
+    bad.K, bad.C = 2048, 16
+    arr2 = (P * 2)(ctypes.pointer(q), ctypes.pointer(bad))
+    assert L.aq_group_workspace_bytes(0, 1, arr2, 2) == 0

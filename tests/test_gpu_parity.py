@@ -169,3 +169,79 @@ def test_device_errors_are_reported():
     with pytest.raises(aq.AqError) as e:
         aq.aq_linear_decode(w, big, torch.ones(65, device="cuda"), ws=aq.workspace(0, 4, w))
     assert e.value.status == -1
+
+
+# ------------------------------------------------------------------ fast quantization path: ties and near-ties
+
+def test_quant_act_exact_ties_everywhere():
+    """amax = 127 * 2^e makes s = 2^e exact, and every (k + 0.5) 2^e is a tie."""
+    rows = []
+    for e in (-6, 0, 3):
+        ks = np.arange(0, 127)
+        vals = np.concatenate([(ks + 0.5), -(ks + 0.5), [127.0]]) * 2.0 ** e
+        vals = np.concatenate([vals, np.zeros(256 - vals.size)])
+        rows.append(vals)
+    x = synth.f32_to_bf16_bits(np.array(rows, np.float32))
+    xq, sx = aq.aq_quant_act(dev_bf16(x))
+    xq_ref, sx_ref = oracle.quant_act(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(sx.cpu().numpy(), sx_ref)
+
+
+def test_quant_act_million_random_elements():
+    x = synth.activations(256, 4096, (31337,), outlier_frac=0.01)
+    xq, sx = aq.aq_quant_act(dev_bf16(x))
+    xq_ref, sx_ref = oracle.quant_act(x)
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)
+    assert np.array_equal(sx.cpu().numpy(), sx_ref)
+
+
+# ------------------------------------------------------------------ shared-input groups
+
+def _group_case(shapes, M, seed, phase, bN=128, frac8=0.25):
+    ps = [synth.projection_inputs(N, K, bN, 128, frac8, (seed, g)) for g, (N, K) in enumerate(shapes)]
+    ws = [aq.aq_pack(*dev_projection(p), bN, 128) for p in ps]
+    x = synth.activations(M, shapes[0][1], (seed, 9), outlier_frac=0.01)
+    return ps, ws, x
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 9, 24, 64])
+def test_group_decode_matches_separate_calls_and_oracle(M):
+    shapes = [(768, 1024), (256, 1024), (256, 1024)]
+    ps, ws, x = _group_case(shapes, M, 1000 + M, aq.AQ_PHASE_DECODE)
+    xd = dev_bf16(x)
+    grp = aq.Group(ws, aq.AQ_PHASE_DECODE, M)
+    outs = [torch.empty((M, N), device="cuda") for N, _ in shapes]
+    biases = [torch.linspace(-1, 1, N, device="cuda") for N, _ in shapes]
+    grp(xd, outs, bias=biases)
+    xq, sx = aq.aq_quant_act(xd)
+    for g, (p, w) in enumerate(zip(ps, ws)):
+        sep = aq.aq_linear_decode(w, xq, sx, bias=biases[g])
+        assert torch.equal(outs[g], sep), g
+        assert_output_close(outs[g], oracle_linear(p, x, bias=biases[g].cpu().numpy()))
+    aq.check_all_workspaces()
+    rc, _ = aq.aq_workspace_status(grp.ws)
+    assert rc == 0
+
+
+@pytest.mark.parametrize("M", [1, 300])
+def test_group_prefill_matches_oracle(M):
+    shapes = [(512, 768), (384, 768)]
+    ps, ws, x = _group_case(shapes, M, 1100 + M, aq.AQ_PHASE_PREFILL, bN=64, frac8=0.4)
+    grp = aq.Group(ws, aq.AQ_PHASE_PREFILL, M)
+    outs = [torch.empty((M, N), device="cuda", dtype=torch.bfloat16) for N, _ in shapes]
+    grp(dev_bf16(x), outs)
+    for p, o in zip(ps, outs):
+        assert_output_close(o, oracle_linear(p, x))
+    rc, _ = aq.aq_workspace_status(grp.ws)
+    assert rc == 0
+
+
+def test_group_rejects_mismatched_inputs():
+    ps, ws, x = _group_case([(256, 512), (256, 512)], 4, 1200, aq.AQ_PHASE_DECODE)
+    p2 = synth.projection_inputs(256, 384, 128, 128, 0.5, (1201,))
+    w2 = aq.aq_pack(*dev_projection(p2), 128, 128)
+    with pytest.raises(ValueError):
+        aq.Group([ws[0], w2], aq.AQ_PHASE_DECODE, 4)
+    with pytest.raises(ValueError):
+        aq.Group(ws, aq.AQ_PHASE_DECODE, 65)

@@ -21,7 +21,7 @@ AQ_PHASE_DECODE, AQ_PHASE_PREFILL = 0, 1
 BUF_NAMES = ("bitmap", "row_off4", "row_off8", "tile_idx", "w4", "w8", "scales")
 EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "aq_quant_act",
             "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
-            "aq_workspace_status")
+            "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status")
 
 
 class AqError(RuntimeError):
@@ -68,6 +68,12 @@ def lib():
                       c_void_p]
     L.aq_debug_tile_partials.restype = c_int
     L.aq_debug_tile_partials.argtypes = [P, c_void_p, c_int, c_int, c_void_p, c_void_p, c_size_t, c_void_p]
+    L.aq_linear_group.restype = c_int
+    L.aq_linear_group.argtypes = [c_int, ctypes.POINTER(P), c_int, c_void_p, c_int, c_int, ctypes.POINTER(c_void_p),
+                                  ctypes.POINTER(c_void_p), ctypes.POINTER(c_int), c_int, c_void_p, c_size_t,
+                                  c_void_p]
+    L.aq_group_workspace_bytes.restype = c_size_t
+    L.aq_group_workspace_bytes.argtypes = [c_int, c_int, ctypes.POINTER(P), c_int]
     L.aq_workspace_status.restype = c_int
     L.aq_workspace_status.argtypes = [c_void_p, c_void_p, ctypes.POINTER(c_int)]
     _lib = L
@@ -209,6 +215,44 @@ def aq_linear_prefill(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=t
     """Prefill-phase y (tensor-core INT8 path), any M >= 1."""
     return _linear(lib().aq_linear_prefill, "aq_linear_prefill", AQ_PHASE_PREFILL, w, xq, sx, bias, out, out_dtype,
                    ws)
+
+
+class Group:
+    """Projections sharing one input (q/k/v or gate/up), run by aq_linear_group."""
+
+    def __init__(self, weights, phase: int, M: int):
+        self.weights = list(weights)
+        self.phase, self.M = phase, M
+        G = len(self.weights)
+        P = ctypes.POINTER(AqPackedStruct)
+        self._w = (P * G)(*[ctypes.pointer(w.struct) for w in self.weights])
+        need = int(lib().aq_group_workspace_bytes(phase, M, self._w, G))
+        if need == 0:
+            raise ValueError("invalid projection group")
+        self.ws = torch.zeros(need, dtype=torch.uint8, device=self.weights[0].device)
+
+    def __call__(self, x: torch.Tensor, outs, bias=None, ws=None):
+        """x bf16 [M][ldx]; outs: one float32 or bfloat16 [M][N_g] tensor per member."""
+        G = len(self.weights)
+        dev = self.weights[0].device
+        if x.dtype != torch.bfloat16 or x.device != dev or x.dim() != 2 or x.stride(1) != 1:
+            raise ValueError("x must be a 2-D bf16 tensor on the weights' device with unit inner stride")
+        if x.shape[0] != self.M or len(outs) != G:
+            raise ValueError("token count or number of outputs does not match the group")
+        dt = outs[0].dtype
+        if dt not in (torch.float32, torch.bfloat16) or any(o.dtype != dt or o.device != dev or o.stride(1) != 1
+                                                             for o in outs):
+            raise ValueError("outputs must share one dtype (float32 or bfloat16) on the weights' device")
+        ys = (ctypes.c_void_p * G)(*[o.data_ptr() for o in outs])
+        lds = (ctypes.c_int * G)(*[o.stride(0) for o in outs])
+        bs = None
+        if bias is not None:
+            bs = (ctypes.c_void_p * G)(*[b.data_ptr() if b is not None else None for b in bias])
+        ws = self.ws if ws is None else ws
+        _check(lib().aq_linear_group(self.phase, self._w, G, x.data_ptr(), x.stride(0), self.M, bs, ys, lds,
+                                     AQ_F32 if dt == torch.float32 else AQ_BF16, ws.data_ptr(), ws.numel(),
+                                     _stream(dev)), "aq_linear_group")
+        return outs
 
 
 def aq_debug_tile_partials(w: PackedWeights, xq: torch.Tensor, phase: int, ws=None) -> torch.Tensor:

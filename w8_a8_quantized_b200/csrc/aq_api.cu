@@ -21,15 +21,16 @@ int validate_packed(const aq_packed* w) {
 
 static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
-// Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, dp4a has room);
-// more tokens on the tensor cores.  Splits over tile columns fill the GPU.
+// Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, one CTA per 16
+// output rows, no split); more tokens on the tensor cores with splits over
+// tile columns to fill the GPU.
 DecodePlan plan_decode(int M, const aq_packed* w) {
   DecodePlan p;
-  if (M <= 8) {
+  if (rows_supported(M, w->K)) {
     p.kernel = 0;
-    p.rows = w->bN;
-    p.blocks = w->R;
-    p.S = std::max(1, std::min(w->C, ceil_div(2 * kNumSMs, p.blocks)));
+    p.rows = 16;
+    p.blocks = w->N / 16;
+    p.S = 1;
   } else {
     p.kernel = 1;
     p.rows = 128;
@@ -43,12 +44,20 @@ static size_t counters_bytes(int blocks) { return ((size_t)blocks * sizeof(int) 
 
 size_t decode_ws_bytes(int M, const aq_packed* w) {
   const DecodePlan p = plan_decode(M, w);
+  if (p.kernel == 0) return kWsHeader;
   size_t b = kWsHeader + counters_bytes(p.blocks);
   if (p.S > 1) b += (size_t)p.S * M * w->N * sizeof(float);
   return b;
 }
 
 size_t prefill_ws_bytes(int /*M*/, const aq_packed* w) { return kWsHeader + counters_bytes(w->R); }
+
+DecodeProj decode_proj(const aq_packed* w, const float* bias, void* y, int ldy) {
+  DecodeProj d;
+  d.bitmap = w->bitmap; d.tile_idx = w->tile_idx; d.w4 = w->w4; d.w8 = w->w8; d.scales = w->scales;
+  d.bias = bias; d.y = y; d.N = w->N; d.bN = w->bN; d.ldy = ldy; d.blocks = w->N / 16;
+  return d;
+}
 
 }  // namespace aq
 
@@ -115,9 +124,13 @@ extern "C" int aq_linear_decode(const aq_packed* w, const int8_t* xq, const floa
   if (M > kMaxDecodeM) return AQ_ERR_ARG;
   if (!ws || ws_bytes < decode_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const DecodePlan p = plan_decode(M, w);
-  cudaError_t e = p.kernel == 0 ? launch_decode_simt(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, st)
-                                : launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_DECODE, st);
+  cudaError_t e;
+  if (plan_decode(M, w).kernel == 0) {
+    const DecodeProj d = decode_proj(w, bias, y, ldy);
+    e = launch_decode_rows(&d, 1, w->K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+  } else {
+    e = launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_DECODE, st);
+  }
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
 }
 
@@ -141,10 +154,89 @@ extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int 
   if (!ws || ws_bytes < kWsHeader) return AQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (phase == AQ_PHASE_DECODE && plan_decode(M, w).kernel == 0)
-    e = launch_decode_simt(w, xq, nullptr, M, nullptr, nullptr, AQ_F32, w->N, ws, P, st);
-  else
+  if (phase == AQ_PHASE_DECODE && plan_decode(M, w).kernel == 0) {
+    const DecodeProj d = decode_proj(w, nullptr, nullptr, w->N);
+    e = launch_decode_rows(&d, 1, w->K, nullptr, 0, xq, nullptr, M, AQ_F32, P, ws, st);
+  } else
     e = launch_tc(w, xq, nullptr, M, nullptr, nullptr, AQ_F32, w->N, ws, P, phase, st);
+  return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- shared-input groups (App. E.4)
+static int check_group(int phase, const aq_packed* const* w, int G, const uint16_t* x, int ldx, int M) {
+  if (!w || G < 1 || G > kMaxGroup || !x || M < 1) return AQ_ERR_ARG;
+  if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return AQ_ERR_ARG;
+  if (phase == AQ_PHASE_DECODE && M > kMaxDecodeM) return AQ_ERR_ARG;
+  for (int g = 0; g < G; ++g) {
+    int rc = validate_packed(w[g]);
+    if (rc != AQ_OK) return rc;
+    if (w[g]->K != w[0]->K) return AQ_ERR_SHAPE;
+  }
+  const int K = w[0]->K;
+  if (ldx < K || ldx % 8 || ((uintptr_t)x & 15)) return AQ_ERR_ARG;
+  return AQ_OK;
+}
+
+static bool group_fused(int phase, const aq_packed* const* w, int G, int M) {
+  return phase == AQ_PHASE_DECODE && rows_supported(M, w[0]->K) && rows_fusable(M, w[0]->K);
+  (void)G;
+}
+
+static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+static size_t group_ws_bytes(int phase, int M, const aq_packed* const* w, int G) {
+  if (group_fused(phase, w, G, M)) return kWsHeader;
+  size_t lin = 0;
+  for (int g = 0; g < G; ++g)
+    lin = std::max(lin, phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w[g]) : prefill_ws_bytes(M, w[g]));
+  // the linear workspace (header first), then the prepared activations
+  return align256(lin) + align256((size_t)M * w[0]->K) + align256((size_t)M * sizeof(float));
+}
+
+extern "C" size_t aq_group_workspace_bytes(int phase, int M, const aq_packed* const* w, int G) {
+  if (!w || G < 1 || G > kMaxGroup || M < 1) return 0;
+  if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return 0;
+  if (phase == AQ_PHASE_DECODE && M > kMaxDecodeM) return 0;
+  for (int g = 0; g < G; ++g)
+    if (validate_packed(w[g]) != AQ_OK || w[g]->K != w[0]->K) return 0;
+  return group_ws_bytes(phase, M, w, G);
+}
+
+extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, const uint16_t* x, int ldx, int M,
+                               const float* const* bias, void* const* y, const int* ldy, int ydtype, void* ws,
+                               size_t ws_bytes, void* stream) {
+  int rc = check_group(phase, w, G, x, ldx, M);
+  if (rc != AQ_OK) return rc;
+  if (!y || !ldy || (ydtype != AQ_F32 && ydtype != AQ_BF16)) return AQ_ERR_ARG;
+  for (int g = 0; g < G; ++g)
+    if (!y[g] || ldy[g] < w[g]->N) return AQ_ERR_ARG;
+  if (!ws || ws_bytes < group_ws_bytes(phase, M, w, G)) return AQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int K = w[0]->K;
+  cudaError_t e = cudaSuccess;
+  if (group_fused(phase, w, G, M)) {
+    DecodeProj d[kMaxGroup];
+    for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
+    e = launch_decode_rows(d, G, K, x, ldx, nullptr, nullptr, M, ydtype, nullptr, ws, st);
+    return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+  }
+  // prepare the shared input once, then run every member on it
+  size_t lin = 0;
+  for (int g = 0; g < G; ++g)
+    lin = std::max(lin, phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w[g]) : prefill_ws_bytes(M, w[g]));
+  char* base = static_cast<char*>(ws);
+  int8_t* xq = reinterpret_cast<int8_t*>(base + align256(lin));
+  float* sx = reinterpret_cast<float*>(base + align256(lin) + align256((size_t)M * K));
+  e = launch_quant_act(x, M, K, ldx, xq, sx, st);
+  for (int g = 0; e == cudaSuccess && g < G; ++g) {
+    const float* b = bias ? bias[g] : nullptr;
+    if (phase == AQ_PHASE_DECODE && plan_decode(M, w[g]).kernel == 0) {
+      const DecodeProj d = decode_proj(w[g], b, y[g], ldy[g]);
+      e = launch_decode_rows(&d, 1, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+    } else {
+      e = launch_tc(w[g], xq, sx, M, b, y[g], ydtype, ldy[g], ws, nullptr, phase, st);
+    }
+  }
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
 }
 

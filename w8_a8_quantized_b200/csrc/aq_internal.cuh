@@ -8,6 +8,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "../../include/aq.h"
 
@@ -37,6 +38,26 @@ inline bool geometry_ok(int N, int K, int bN, int bK) {
 
 int validate_packed(const aq_packed* w);  // AQ_OK or an error status
 
+// One projection as seen by the CUDA-core decode kernel (a group of up to
+// kMaxGroup projections sharing one input runs as a single launch).
+constexpr int kMaxGroup = 3;
+constexpr int kRowsMaxM = 8;                   // tokens handled by the CUDA-core decode kernel
+constexpr size_t kFusedMaxBytes = 64 * 1024;   // shared memory for fused activation codes
+struct DecodeProj {
+  const uint8_t* bitmap;
+  const int32_t* tile_idx;
+  const uint8_t* w4;
+  const int8_t* w8;
+  const uint16_t* scales;
+  const float* bias;
+  void* y;
+  int N, bN, ldy, blocks;
+};
+bool rows_supported(int M, int K);
+bool rows_fusable(int M, int K);
+cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
+                               const float* sx, int M, int ydtype, int32_t* P, void* ws, cudaStream_t st);
+
 // Split-K plan of the decode kernels (a pure function of the geometry, so
 // the workspace size and the launch agree).
 struct DecodePlan {
@@ -53,8 +74,6 @@ size_t prefill_ws_bytes(int M, const aq_packed* w);
 cudaError_t launch_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, cudaStream_t st);
 cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, const aq_packed* out,
                                 const uint8_t* map_dev, int* err_dev, cudaStream_t st);
-cudaError_t launch_decode_simt(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
-                               void* y, int ydtype, int ldy, void* ws, int32_t* P, cudaStream_t st);
 cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
                       int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st);
 
@@ -125,6 +144,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16), no multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -166,6 +193,16 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 consecutive 32-bit columns, every value = v.
+__device__ __forceinline__ void tmem_st16_const(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
 
 // 32 lanes x 16 consecutive 32-bit columns: thread t of the warp receives lane
 // (warp quadrant * 32 + t), columns col .. col+15.
@@ -210,6 +247,69 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
+// ---- per-token INT8 activation quantization (shared by every kernel that prepares activations)
+__device__ __forceinline__ float abs_max8(const uint4& v, float m) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, bf16_bits_to_float(w[i] & 0x7FFFu));
+    m = fmaxf(m, bf16_bits_to_float((w[i] >> 16) & 0x7FFFu));
+  }
+  return m;
+}
+
+// s = max(amax / 127, 1e-12) in fp64 (eq. 6 floor).
+__device__ __forceinline__ double act_scale(float amax) {
+  double s = static_cast<double>(amax) / 127.0;
+  return s < 1e-12 ? 1e-12 : s;
+}
+
+// clamp(rint(x / s), -127, 127) with x / s rounded in fp64, as the oracle does.
+// Fast path: t = x * fl32(1/s) is within |x/s| * 2^-23 <= 1.6e-5 of x / s
+// (|x / s| <= 127); when t is more than 3e-5 away from the nearest half-integer
+// the exact quotient, and its fp64 rounding, round to the same integer as t.
+// Otherwise (ties and near-ties) the fp64 division decides.
+__device__ __forceinline__ int quant_code(float x, double s, float r32) {
+  const float t = x * r32;
+  const float k = rintf(t);
+  if (0.5f - fabsf(t - k) > 3.0e-5f) return static_cast<int>(fminf(fmaxf(k, -127.f), 127.f));
+  const double q = rint(static_cast<double>(x) / s);
+  return static_cast<int>(fmin(fmax(q, -127.0), 127.0));
+}
+
+__device__ __forceinline__ uint2 quantize8(const uint4& v, double s, float r32) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t out[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c0 = quant_code(bf16_bits_to_float(w[2 * h] & 0xFFFFu), s, r32);
+    const int c1 = quant_code(bf16_bits_to_float(w[2 * h] >> 16), s, r32);
+    const int c2 = quant_code(bf16_bits_to_float(w[2 * h + 1] & 0xFFFFu), s, r32);
+    const int c3 = quant_code(bf16_bits_to_float(w[2 * h + 1] >> 16), s, r32);
+    out[h] = (uint32_t)(c0 & 0xFF) | ((uint32_t)(c1 & 0xFF) << 8) | ((uint32_t)(c2 & 0xFF) << 16) |
+             ((uint32_t)(c3 & 0xFF) << 24);
+  }
+  return make_uint2(out[0], out[1]);
+}
+
 #endif  // __CUDACC__
+
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel on the stream finishes; it must call pdl_wait() before it
+// reads anything an earlier kernel wrote and before its first global write.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 }  // namespace aq

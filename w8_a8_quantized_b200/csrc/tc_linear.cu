@@ -43,8 +43,8 @@ struct TcShape {
   static constexpr int kB = NT * kTileK;         // swizzled INT8 activation block
   static constexpr int kStageBytes = kA + kB + kStg;
   static constexpr int kStages = NT >= 256 ? 3 : (NT >= 128 ? 4 : 6);
-  static constexpr int kEpiWarps = NT > 128 ? 8 : 4;
-  static constexpr int kCols = NT / (kEpiWarps / 4);  // accumulator columns per epilogue thread
+  static constexpr int kEpiWarps = NT > 64 ? 4 * (NT / 64) : 4;  // 4 warps (one per lane quadrant) per 64 columns
+  static constexpr int kCols = NT / (kEpiWarps / 4);             // accumulator columns per epilogue thread (<= 64)
   static constexpr int kThreads = 128 + 32 * kEpiWarps;
   static constexpr int kTmemCols = 2 * NT <= 32 ? 32 : 2 * NT <= 64 ? 64 : 2 * NT <= 128 ? 128 : 2 * NT <= 256 ? 256 : 512;
   static constexpr int kBufStride = kTmemCols / 2;  // column offset of accumulator buffer 1
@@ -56,6 +56,9 @@ struct TcShape {
   static_assert((4 * kStages + 5) * 8 + 16 <= kBarBytes, "barrier area");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
+
+constexpr uint32_t kAccBias = 0x4B400000u;  // fp32 bit pattern of 12582912 = 1.5 * 2^23
+constexpr float kAccBiasF = 12582912.0f;
 
 struct TcArgs {
   const uint8_t* bitmap;
@@ -105,13 +108,13 @@ __device__ __forceinline__ void tile_kinds(const TcArgs& a, int rb, int j, int& 
   }
 }
 
-// Sign-extend 8 nibbles (low nibble = even k) into 8 INT8 bytes.
-__device__ __forceinline__ uint2 expand8(uint32_t v) {
-  const uint32_t lo = v & 0x0F0F0F0Fu, hi = (v >> 4) & 0x0F0F0F0Fu;
-  uint32_t a = __byte_perm(lo, hi, 0x5140), b = __byte_perm(lo, hi, 0x7362);
-  a = ((a ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;  // per byte: u -> u < 8 ? u : u - 16
-  b = ((b ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-  return make_uint2(a, b);
+// 8 nibbles (low nibble = even k) -> 8 INT8 bytes holding 16 * q in k order.
+// A nibble placed in the high half of a byte with a zero low half IS the
+// two's-complement byte 16 q, so no sign extension is needed; the MMA then
+// yields 16 P for INT4 tiles and the epilogue scales by sw / 16 (exact).
+__device__ __forceinline__ uint2 expand8_x16(uint32_t v) {
+  const uint32_t lo = (v << 4) & 0xF0F0F0F0u, hi = v & 0xF0F0F0F0u;
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
 __device__ __forceinline__ void store_y(void* y, int ydtype, size_t idx, float v) {
@@ -174,6 +177,7 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_launch_dependents();
 
   auto fail = [&](int info) {
     *abort_flag = 1;
@@ -183,6 +187,7 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      pdl_wait();  // activations come from an earlier kernel
       uint32_t g = 0, stg_bits = 0, stg_used = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
@@ -242,15 +247,16 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
             if (!mbar_wait(&expanded[st], (exp_bits >> st) & 1, abort_flag)) { fail(3); ok = false; break; }
             exp_bits ^= 1u << st;
           }
-          const int ab = kt & 1;
-          if (!mbar_wait(&tmem_empty[ab], ((kt >> 1) & 1) ^ 1, abort_flag)) { fail(4); ok = false; break; }
+          const int ab = kt & 1;  // use kt >> 1 of this buffer waits for the epilogue's release number kt >> 1
+          if (!mbar_wait(&tmem_empty[ab], (kt >> 1) & 1, abort_flag)) { fail(4); ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sw128_desc(smem_u32(stage_a(st)));
           const uint64_t bdesc = sw128_desc(smem_u32(stage_b(st)));
           const uint32_t d = tmem_base + ab * Sh::kBufStride;
+          // the buffer holds the bias kAccBias in every element; all four MMAs accumulate onto it
 #pragma unroll
           for (int k = 0; k < kTileK / 32; ++k)  // K = 32 bytes per instruction: +2 in 16-byte units
-            mma_i8(d, adesc + 2 * k, bdesc + 2 * k, Sh::kIdesc, k > 0 ? 1u : 0u);
+            mma_i8(d, adesc + 2 * k, bdesc + 2 * k, Sh::kIdesc, 1u);
           mma_commit(&empty[st]);
           mma_commit(&tmem_full[ab]);
         }
@@ -281,7 +287,7 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
           for (int q = et; q < a.bN * 4; q += 64) {  // 16-byte source chunks
             const int n = q >> 2, c4 = q & 3;
             const uint4 v = *reinterpret_cast<const uint4*>(src + n * 64 + c4 * 16);
-            const uint2 e0 = expand8(v.x), e1 = expand8(v.y), e2 = expand8(v.z), e3 = expand8(v.w);
+            const uint2 e0 = expand8_x16(v.x), e1 = expand8_x16(v.y), e2 = expand8_x16(v.z), e3 = expand8_x16(v.w);
             const int kc0 = 2 * c4, kc1 = 2 * c4 + 1;  // logical 16-byte chunks of the 128-byte row
             *reinterpret_cast<uint4*>(dst + n * 128 + ((kc0 ^ (n & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
             *reinterpret_cast<uint4*>(dst + n * 128 + ((kc1 ^ (n & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
@@ -299,6 +305,21 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
     const int cg = ew >> 2;          // column group
     const int row = 32 * quad + lane;  // row inside the 128-row block
     const int sub = row / a.bN, nl = row % a.bN;
+    pdl_wait();  // outputs and workspace may still be in use by an earlier kernel
+    // Bias both accumulator buffers: an INT32 sum P accumulated onto 0x4B400000
+    // reads, as an fp32 bit pattern, exactly 12582912 + P for |P| < 2^22, so one
+    // fp32 subtraction converts it (no int -> float conversion instruction).
+    {
+      const uint32_t lane_base = tmem_base + ((uint32_t)(32 * quad) << 16) + cg * Sh::kCols;
+#pragma unroll
+      for (int ab = 0; ab < 2; ++ab)
+#pragma unroll
+        for (int c16 = 0; c16 < Sh::kCols / 16; ++c16) tmem_st16_const(lane_base + ab * Sh::kBufStride + c16 * 16, kAccBias);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&tmem_empty[0]);
+      mbar_arrive(&tmem_empty[1]);
+    }
     uint32_t kt = 0, sync_phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
@@ -312,8 +333,12 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
       for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
       for (int j = x.j0; j < x.j1; ++j, ++kt) {
         const int ab = kt & 1;
-        const float sw =
-            rvalid ? __half2float(__ushort_as_half(__ldg(a.scales + ((size_t)r * a.C + j) * a.bN + nl))) : 0.f;
+        const int tt = r * a.C + j;
+        // INT4 tiles were multiplied by 16 during expansion
+        const bool t4 = rvalid && ((__ldg(a.bitmap + (tt >> 3)) >> (tt & 7)) & 1);
+        const float sw = rvalid ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)tt * a.bN + nl))) *
+                                      (t4 ? 0.0625f : 1.0f)
+                                : 0.f;
         // warp-uniform outcome: the tensor-memory loads below are warp-collective
         if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[ab], (kt >> 1) & 1, abort_flag))) {
           fail(6);
@@ -327,17 +352,23 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
           uint32_t v[16];
           tmem_ld16(taddr + c16 * 16, v);
           tmem_wait_ld();
+          tmem_st16_const(taddr + c16 * 16, kAccBias);  // re-bias for the buffer's next use
           if (a.P != nullptr) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int m = mcol0 + c16 * 16 + i;
-              if (rvalid && m < a.M) a.P[((size_t)m * a.N + n) * a.C + j] = (int)v[i];
+              if (rvalid && m < a.M) {
+                const int p16 = (int)(v[i] - kAccBias);
+                a.P[((size_t)m * a.N + n) * a.C + j] = t4 ? (p16 >> 4) : p16;
+              }
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[c16 * 16 + i] = fmaf((float)(int)v[i], sw, acc[c16 * 16 + i]);
+            for (int i = 0; i < 16; ++i)
+              acc[c16 * 16 + i] = fmaf(__uint_as_float(v[i]) - kAccBiasF, sw, acc[c16 * 16 + i]);
           }
         }
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&tmem_empty[ab]);
       }
@@ -444,8 +475,7 @@ cudaError_t launch_nt(const aq_packed* w, const int8_t* xq, TcArgs a, int grid, 
   if (w->T4 > 0 && !make_map(&m4, w->w4, kTileK / 2, (uint64_t)w->T4 * w->bN, kTileK / 2, w->bN, false))
     return cudaErrorInvalidValue;
   if (!make_map(&mx, xq, w->K, a.M, kTileK, NT, true)) return cudaErrorInvalidValue;
-  tc_linear_kernel<NT><<<grid, Sh::kThreads, Sh::kSmemBytes, st>>>(m8, m4, mx, a);
-  return cudaGetLastError();
+  return launch_pdl(tc_linear_kernel<NT>, dim3(grid), dim3(Sh::kThreads), (size_t)Sh::kSmemBytes, st, m8, m4, mx, a);
 }
 
 }  // namespace
