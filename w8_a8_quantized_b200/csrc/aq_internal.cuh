@@ -121,13 +121,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete.  Returns false when
 // `abort` became nonzero or the time limit passed; never spins unbounded.
+// Reading %globaltimer costs hundreds of nanoseconds, so the clock (and the
+// abort flag) are checked only every 256 unsuccessful polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  while (true) {
+  unsigned long long t0 = 0;
+  for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    if ((n & 255u) == 0) {
+      if (*abort) return false;
+      const unsigned long long now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitTimeoutNs) return false;
+    }
   }
 }
 
@@ -264,15 +270,19 @@ __device__ __forceinline__ double act_scale(float amax) {
   return s < 1e-12 ? 1e-12 : s;
 }
 
+// r32 for quant_code: fp32 reciprocal of fp32(s), relative error <= 2 * 2^-24.
+__device__ __forceinline__ float act_recip(double s) { return __frcp_rn(static_cast<float>(s)); }
+
 // clamp(rint(x / s), -127, 127) with x / s rounded in fp64, as the oracle does.
-// Fast path: t = x * fl32(1/s) is within |x/s| * 2^-23 <= 1.6e-5 of x / s
-// (|x / s| <= 127); when t is more than 3e-5 away from the nearest half-integer
-// the exact quotient, and its fp64 rounding, round to the same integer as t.
-// Otherwise (ties and near-ties) the fp64 division decides.
+// Fast path: t = x * r32 carries at most three roundings of 2^-24 each
+// (fp32(s), the reciprocal, the product), so |t - x/s| <= 127 * 3 * 2^-24
+// < 2.3e-5 (|x / s| <= 127).  When t is more than 4e-5 away from the nearest
+// half-integer the exact quotient, and its fp64 rounding, round to the same
+// integer as t; otherwise (ties and near-ties) the fp64 division decides.
 __device__ __forceinline__ int quant_code(float x, double s, float r32) {
   const float t = x * r32;
   const float k = rintf(t);
-  if (0.5f - fabsf(t - k) > 3.0e-5f) return static_cast<int>(fminf(fmaxf(k, -127.f), 127.f));
+  if (0.5f - fabsf(t - k) > 4.0e-5f) return static_cast<int>(fminf(fmaxf(k, -127.f), 127.f));
   const double q = rint(static_cast<double>(x) / s);
   return static_cast<int>(fmin(fmax(q, -127.0), 127.0));
 }

@@ -1,78 +1,74 @@
 // Decode-phase linear layers on the CUDA cores for a few tokens.
 //
-// AlignQuant, Sec. 3.3 "Decode parallelism" and App. E.3: the kernel streams
-// the packed tiles from HBM, forms INT8 operands on chip, takes per-tile INT32
-// dot products and rescales each by its activation and weight scales before
-// FP32 accumulation (eq. 19).  Sec. 3.3 "Shared activation preparation" and
+// AlignQuant, Sec. 3.3 "Decode parallelism" and App. E.3: the kernel loads the
+// packed tiles from HBM, forms INT8 operands on chip, takes per-tile INT32 dot
+// products and rescales each by its activation and weight scales before FP32
+// accumulation (eq. 19).  Sec. 3.3 "Shared activation preparation" and
 // App. E.4: projections that read the same input (q/k/v, gate/up) run as one
 // launch over their concatenated output rows, and the activation quantization
 // can be fused into that launch so each CTA prepares the input from bf16.
 //
-// Work split: one CTA owns kRows = 16 consecutive output rows of one
+// Work split: one CTA owns kRows = 32 consecutive output rows of one
 // projection and ALL of its input tiles, so there is no cross-CTA reduction.
-// The 16-row slice of a tile is contiguous in the packed buffers (2 KB for
-// INT8, 1 KB for INT4, plus 32 B of row scales), so thread 0 streams slices
-// into a shared-memory ring with one asynchronous bulk copy each
-// (cp.async.bulk, completion counted on an mbarrier) and keeps up to
-// kMaxStages slices in flight per CTA without spending registers.  The copies
-// of the first ring fill are issued before griddepcontrol.wait: weights never
-// depend on an earlier kernel, so a launch streams while its predecessor ends.
+// The CTA has KG groups of 64 threads (KG = 1..8, chosen so the launch keeps
+// about 16 warps per SM busy); group kg takes tile columns kg, kg + KG, ...
+// In a group, thread t owns row t / 2 and half h = t % 2 of every tile row:
+// input columns [64h, 64h + 64), i.e. 64 contiguous bytes of an INT8 tile row
+// (four 16-byte loads) or 32 bytes of an INT4 tile row (two).  A warp reads 16
+// whole tile rows per load step: 2 KB (INT8) or 1 KB (INT4) contiguous.  Big
+// per-thread pieces keep the instruction count per weight byte low: at HBM
+// rate the SM issue rate, not memory, is what a finer split runs out of.
 //
-// Thread t owns row t / 8 and, in every tile, the 16 input columns
-// [16c, 16c + 16) with c = t % 8; a warp reads 4 whole slice rows per
-// shared-memory access (512 contiguous bytes of an INT8 slice, 256 of INT4).
-// INT4 nibbles are unpacked in registers: (v & 0x0F0F0F0F) ^ 0x08080808 gives
-// the even-k codes plus 8 as unsigned bytes, the shifted word the odd-k codes;
-// byte permutes restore k order, an unsigned x signed dp4a against the
-// activation bytes gives sum((q + 8) x), and 8 x sum(x) is subtracted.  The 8
-// lanes of a row keep separate FP32 sums of (exact lane partial) x (tile
-// scale) and are combined with shuffles once, after the last tile.
+// Memory pipeline: each thread keeps its next kRing tiles in flight in a ring
+// of registers (the loop is unrolled kRing times, a load's destination is read
+// kRing tiles later, the register scoreboard is the only wait).  Tile
+// addresses, INT4 labels and the CTA's fp16 row scales are staged in shared
+// memory once, and the first ring of loads is issued before
+// griddepcontrol.wait: weights never depend on an earlier kernel, so a launch
+// streams while its predecessor finishes.
 //
-// Every mbarrier wait is bounded; a wait that gives up records AQ_ERR_TIMEOUT
-// in the workspace, the CTA stops consuming, and thread 0 waits (bounded) for
-// the copies it issued before the CTA exits.
+// INT4 nibbles are unpacked in registers without sign extension: a nibble in
+// the high half of a byte with a zero low half IS the two's-complement byte
+// 16 q, so (v << 4) & 0xF0F0F0F0 holds 16 q of the even k of a word and
+// v & 0xF0F0F0F0 of the odd k.  A dp4a against the activation bytes of the
+// even / odd k gives 16 x the exact product, and the tile scale is divided by
+// 16 (exact).  The fused path stores the activation codes twice in shared
+// memory: in k order (for INT8 tiles) and with even and odd k split per
+// 8-column group (for INT4 tiles); the pre-quantized path permutes on the fly.
+// The 2 lanes of a row keep FP32 sums of (exact lane partial) x (tile scale)
+// and are combined once, after the last tile, then the KG groups in order.
 #include "aq_internal.cuh"
 
 namespace aq {
 namespace {
 
-constexpr int kRows = 16;
-constexpr int kThreads = kRows * 8;
-constexpr int kWarps = kThreads / 32;
-constexpr int kMaxC = 256;                       // input tiles per row (K <= 32768)
-constexpr int kMaxStages = 24;                   // slices in flight per CTA
-constexpr int kSliceW = kRows * kTileK;          // bytes of the largest (INT8) slice
-constexpr int kStageBytes = kSliceW + 2 * kRows; // slice + fp16 row scales
+constexpr int kRows = 32;
+constexpr int kGroupThreads = kRows * 2;  // threads of one tile group
+constexpr int kMaxKG = 8;
+constexpr int kMaxThreads = kGroupThreads * kMaxKG;
+constexpr int kMaxC = 256;  // input tiles per row (K <= 32768)
+constexpr int kRing = 4;    // tiles in flight per thread
 
 struct RowsArgs {
   DecodeProj p[kMaxGroup];
-  int G, K, C, M, ydtype, NS;
+  int G, K, C, M, ydtype, KG;
   const uint16_t* x;   // bf16 activations [M][ldx] (fused quantization), or null
   int ldx;
   const int8_t* xq;    // pre-quantized activations [M][K], or null
   const float* sx;
   int32_t* P;          // debug: exact tile products [M][N][C] of projection 0
-  void* ws;            // status word
 };
 
-__device__ __forceinline__ int dp4a_ss(int a, int b, int c) { return __dp4a(a, b, c); }
-__device__ __forceinline__ int dp4a_us(uint32_t a, int b, int c) {
-  int d;
-  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
+__device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) { return __dp4a((int)a, (int)b, c); }
 
 // Exact int -> float for |v| < 2^22 with an integer add and a float subtract.
 __device__ __forceinline__ float small_int_to_float(int v) {
   return __int_as_float(v + 0x4B400000) - 12582912.0f;
 }
 
-// Nibble word (8 codes, low nibble = even k) -> two words of (code + 8) bytes in k order.
-__device__ __forceinline__ void nibbles_plus8(uint32_t v, uint32_t& a, uint32_t& b) {
-  const uint32_t lo = (v & 0x0F0F0F0Fu) ^ 0x08080808u, hi = ((v >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-  a = __byte_perm(lo, hi, 0x5140);
-  b = __byte_perm(lo, hi, 0x7362);
-}
+// even-k / odd-k activation bytes of an 8-column group given in k order
+__device__ __forceinline__ uint32_t even_bytes(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x6420); }
+__device__ __forceinline__ uint32_t odd_bytes(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x7531); }
 
 __device__ __forceinline__ void store_out(void* y, int ydtype, size_t idx, float v) {
   if (ydtype == AQ_F32)
@@ -81,14 +77,19 @@ __device__ __forceinline__ void store_out(void* y, int ydtype, size_t idx, float
     reinterpret_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
 }
 
-template <int MT, bool FUSED>
-__global__ void __launch_bounds__(kThreads) decode_rows_kernel(const __grid_constant__ RowsArgs a) {
-  // dynamic: ring [NS][kStageBytes], then (FUSED) codes [M][K] int8 and sx [M] fp32
+struct Piece {  // one thread's share of one tile row: 64 INT8 bytes or 32 INT4 bytes
+  uint4 v[4];
+};
+
+template <int MT, bool FUSED, bool DEBUG>
+__global__ void __launch_bounds__(kMaxThreads) decode_rows_kernel(const __grid_constant__ RowsArgs a) {
+  // dynamic (FUSED only): codes in k order [M][K], codes even/odd split [M][K], sx [M] fp32
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int32_t desc[kMaxC];  // (physical index << 1) | INT4 label, per tile column
-  __shared__ float red[kWarps][MT];
-  __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
-  __shared__ int flags[2];         // [0] abort, [1] stays 0 (drain waits)
+  __shared__ const uint8_t* tile_ptr[kMaxC];                // slice start (row nl0) of every tile column
+  __shared__ __align__(16) uint16_t tile_sw[kMaxC][kRows];  // fp16 row scales of every tile column
+  __shared__ uint32_t tile_is4[kMaxC / 32];                  // INT4 labels, one bit per tile column
+  __shared__ float red[kMaxKG][kRows][MT];
+  __shared__ float redq[kMaxThreads / 32][MT];
 
   int b = blockIdx.x, g = 0;
 #pragma unroll
@@ -98,89 +99,123 @@ __global__ void __launch_bounds__(kThreads) decode_rows_kernel(const __grid_cons
       ++g;
     }
   const DecodeProj& p = a.p[g];
-  const int t = threadIdx.x, c = t & 7, lrow = t >> 3, lane = t & 31;
-  const int bN = p.bN, C = a.C, K = a.K, M = a.M, NS = a.NS;
-  const int row0 = b * kRows;                   // first output row of the CTA (one tile row holds it)
+  const int nthr = blockDim.x, KG = a.KG;
+  const int t = threadIdx.x, kg = t / kGroupThreads, tg = t % kGroupThreads;
+  const int h = tg & 1, lrow = tg >> 1, lane = t & 31;
+  const int bN = p.bN, C = a.C, K = a.K, M = a.M;
+  const int nmine = (C - kg + KG - 1) / KG;  // tile columns of this thread's group
+  const int row0 = b * kRows;                // first output row of the CTA (one tile row holds it)
   const int r = row0 / bN, nl0 = row0 - r * bN;
   const int row = row0 + lrow;
   const int tile0 = r * C;
-  volatile int* abort_flag = &flags[0];
-  volatile int* never_flag = &flags[1];
 
-  if (t == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kWarps);
-    }
-    flags[0] = flags[1] = 0;
-    fence_mbar_init();
-  }
-  for (int j = t; j < C; j += kThreads) {  // tile metadata (independent of earlier kernels)
+  // ---- per-CTA tile table and scales (independent of earlier kernels)
+  for (int w = t; w < (C + 31) / 32; w += nthr) tile_is4[w] = 0u;
+  __syncthreads();
+  for (int j = t; j < C; j += nthr) {
     const int tt = tile0 + j;
     const int is4 = (__ldg(p.bitmap + (tt >> 3)) >> (tt & 7)) & 1;
-    desc[j] = (__ldg(p.tile_idx + tt) << 1) | is4;
+    const size_t pr = (size_t)__ldg(p.tile_idx + tt) * bN + nl0;
+    tile_ptr[j] = is4 ? p.w4 + pr * (kTileK / 2) : reinterpret_cast<const uint8_t*>(p.w8) + pr * kTileK;
+    if (is4) atomicOr(&tile_is4[j >> 5], 1u << (j & 31));
+  }
+  for (int q = t; q < 4 * C; q += nthr) {  // 32 rows x 2 B = four 16-byte pieces per tile column
+    const int j = q >> 2, part = q & 3;
+    *reinterpret_cast<uint4*>(&tile_sw[j][8 * part]) =
+        __ldg(reinterpret_cast<const uint4*>(p.scales + (size_t)(tile0 + j) * bN + nl0 + 8 * part));
   }
   __syncthreads();
   pdl_launch_dependents();
 
-  auto issue = [&](int j) {  // thread 0 only: slice + row scales of tile column j into stage j % NS
-    const int s = j % NS;
-    const int d = desc[j];
-    const size_t pr = (size_t)(d >> 1) * bN + nl0;  // first physical row of the slice
-    const uint32_t bytes = (d & 1) ? kRows * (kTileK / 2) : kRows * kTileK;
-    const void* src = (d & 1) ? (const void*)(p.w4 + pr * (kTileK / 2)) : (const void*)(p.w8 + pr * kTileK);
-    uint8_t* st = smem + (size_t)s * kStageBytes;
-    mbar_arrive_expect_tx(&full[s], bytes + 2 * kRows);
-    bulk_load(st, src, bytes, &full[s]);
-    bulk_load(st + kSliceW, p.scales + (size_t)(tile0 + j) * bN + nl0, 2 * kRows, &full[s]);
+  // ---- this thread's piece of its i-th tile column (j = kg + KG i)
+  auto load = [&](int i, Piece& pc) {
+    const int j = kg + KG * i;
+    const bool is4 = (tile_is4[j >> 5] >> (j & 31)) & 1;
+    if (is4) {
+      const uint4* src = reinterpret_cast<const uint4*>(tile_ptr[j] + lrow * (kTileK / 2) + 32 * h);
+      pc.v[0] = __ldcs(src);
+      pc.v[1] = __ldcs(src + 1);
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(tile_ptr[j] + lrow * kTileK + 64 * h);
+      pc.v[0] = __ldcs(src);
+      pc.v[1] = __ldcs(src + 1);
+      pc.v[2] = __ldcs(src + 2);
+      pc.v[3] = __ldcs(src + 3);
+    }
   };
-  int issued = 0;
-  if (t == 0)
-    for (; issued < NS && issued < C; ++issued) issue(issued);
+  Piece ring[kRing];
+#pragma unroll
+  for (int q = 0; q < kRing; ++q)
+    if (q < nmine) load(q, ring[q]);
 
   pdl_wait();  // activations (and every global write below) depend on earlier kernels
 
-  const int8_t* xs;
+  const int8_t* xs;    // codes in k order
+  const int8_t* xeo;   // codes, even / odd k split per 8 columns (FUSED only)
   const float* sxp;
-  uint8_t* xbuf = smem + (size_t)NS * kStageBytes;
   if constexpr (FUSED) {
-    // per-token absmax over K, then codes into shared memory (same arithmetic as aq_quant_act)
+    // per-token absmax over K, then codes into shared memory (same arithmetic as
+    // aq_quant_act); each thread keeps up to kXv of its activation vectors in registers
+    constexpr int kXv = MT == 1 ? 4 : 2;
     const int nvec = K / 8;
+    const int nwarps = nthr / 32;
     float amax[MT];
+    uint4 xr[MT][kXv];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) amax[m] = 0.f;
-    for (int v = t; v < nvec; v += kThreads) {
+    for (int m = 0; m < MT; ++m) {
+      amax[m] = 0.f;
+      if (m < M) {
+        const uint4* xrow = reinterpret_cast<const uint4*>(a.x + (size_t)m * a.ldx);
 #pragma unroll
-      for (int m = 0; m < MT; ++m)
-        if (m < M) amax[m] = abs_max8(__ldg(reinterpret_cast<const uint4*>(a.x + (size_t)m * a.ldx) + v), amax[m]);
+        for (int q = 0; q < kXv; ++q) {
+          const int v = t + q * nthr;
+          if (v < nvec) {
+            xr[m][q] = __ldg(xrow + v);
+            amax[m] = abs_max8(xr[m][q], amax[m]);
+          }
+        }
+        for (int v = t + kXv * nthr; v < nvec; v += nthr) amax[m] = abs_max8(__ldg(xrow + v), amax[m]);
+      }
     }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax[m] = fmaxf(amax[m], __shfl_xor_sync(0xffffffffu, amax[m], o));
-      if (lane == 0) red[t >> 5][m] = amax[m];
+      if (lane == 0) redq[t >> 5][m] = amax[m];
     }
     __syncthreads();
-    float* sx_s = reinterpret_cast<float*>(xbuf + (size_t)M * K);
+    uint8_t* cbuf = smem;                       // k order
+    uint8_t* ebuf = smem + (size_t)M * K;       // even / odd split
+    float* sx_s = reinterpret_cast<float*>(smem + 2 * (size_t)M * K);
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       if (m >= M) break;
-      float am = red[0][m];
+      float am = redq[lane < nwarps ? lane : 0][m];
 #pragma unroll
-      for (int w = 1; w < kWarps; ++w) am = fmaxf(am, red[w][m]);
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));  // all lanes agree
       const double s = act_scale(am);
-      const float r32 = (float)(1.0 / s);
-      for (int v = t; v < nvec; v += kThreads) {
-        const uint4 xv = __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)m * a.ldx) + v);
-        *reinterpret_cast<uint2*>(xbuf + (size_t)m * K + 8 * v) = quantize8(xv, s, r32);
+      const float r32 = act_recip(s);
+      const uint4* xrow = reinterpret_cast<const uint4*>(a.x + (size_t)m * a.ldx);
+      auto put = [&](int v, const uint4& xv) {
+        const uint2 q = quantize8(xv, s, r32);  // 8 codes of columns 8v .. 8v+7
+        *reinterpret_cast<uint2*>(cbuf + (size_t)m * K + 8 * v) = q;
+        *reinterpret_cast<uint2*>(ebuf + (size_t)m * K + 8 * v) = make_uint2(even_bytes(q.x, q.y), odd_bytes(q.x, q.y));
+      };
+#pragma unroll
+      for (int q = 0; q < kXv; ++q) {
+        const int v = t + q * nthr;
+        if (v < nvec) put(v, xr[m][q]);
       }
+      for (int v = t + kXv * nthr; v < nvec; v += nthr) put(v, __ldg(xrow + v));
       if (t == 0) sx_s[m] = (float)s;
     }
     __syncthreads();
-    xs = reinterpret_cast<const int8_t*>(xbuf);
+    xs = reinterpret_cast<const int8_t*>(cbuf);
+    xeo = reinterpret_cast<const int8_t*>(ebuf);
     sxp = sx_s;
   } else {
     xs = a.xq;
+    xeo = nullptr;
     sxp = a.sx;
   }
 
@@ -188,116 +223,117 @@ __global__ void __launch_bounds__(kThreads) decode_rows_kernel(const __grid_cons
 #pragma unroll
   for (int m = 0; m < MT; ++m) acc[m] = 0.f;
 
-  bool ok = true;
-  for (int j = 0; j < C; ++j) {
-    const int s = j % NS;
-    const uint32_t ph = (uint32_t)(j / NS) & 1u;
-    if (!mbar_wait(&full[s], ph, abort_flag)) {
-      *abort_flag = 1;
-      record_error(a.ws, AQ_ERR_TIMEOUT, 20);
-      ok = false;
-      break;
-    }
-    const uint8_t* st = smem + (size_t)s * kStageBytes;
-    const bool is4 = desc[j] & 1;
-    const float sw = __half2float(*reinterpret_cast<const __half*>(st + kSliceW + 2 * lrow));
-    uint32_t w0, w1, w2, w3;
-    if (is4) {
-      const uint2 v = *reinterpret_cast<const uint2*>(st + lrow * (kTileK / 2) + 8 * c);
-      nibbles_plus8(v.x, w0, w1);
-      nibbles_plus8(v.y, w2, w3);
-    } else {
-      const uint4 v = *reinterpret_cast<const uint4*>(st + lrow * kTileK + 16 * c);
-      w0 = v.x; w1 = v.y; w2 = v.z; w3 = v.w;
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with stage s
+  auto tile = [&](int i, const Piece& pc) {
+    const int j = kg + KG * i;
+    const bool is4 = (tile_is4[j >> 5] >> (j & 31)) & 1;
+    const float sw = __half2float(__ushort_as_half(tile_sw[j][lrow])) * (is4 ? 0.0625f : 1.0f);
+    const size_t xoff = (size_t)j * kTileK + 64 * h;  // this thread's 64 activation columns
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       if (m >= M) break;
-      const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)m * K + (size_t)j * kTileK + 16 * c);
-      int part;
+      int part = 0;
       if (is4) {
-        int xsum = dp4a_ss((int)xv.x, 0x01010101, 0);
-        xsum = dp4a_ss((int)xv.y, 0x01010101, xsum);
-        xsum = dp4a_ss((int)xv.z, 0x01010101, xsum);
-        xsum = dp4a_ss((int)xv.w, 0x01010101, xsum);
-        part = dp4a_us(w0, (int)xv.x, -8 * xsum);
-        part = dp4a_us(w1, (int)xv.y, part);
-        part = dp4a_us(w2, (int)xv.z, part);
-        part = dp4a_us(w3, (int)xv.w, part);
+        const uint32_t wv[8] = {pc.v[0].x, pc.v[0].y, pc.v[0].z, pc.v[0].w,
+                                pc.v[1].x, pc.v[1].y, pc.v[1].z, pc.v[1].w};
+        uint4 xe[4];
+        if constexpr (FUSED) {
+          const uint4* xp = reinterpret_cast<const uint4*>(xeo + (size_t)m * K + xoff);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) xe[q] = xp[q];  // (even, odd) word pairs of 8-column groups
+        } else {
+          const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)m * K + xoff);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 n = __ldg(xp + q);
+            xe[q] = make_uint4(even_bytes(n.x, n.y), odd_bytes(n.x, n.y), even_bytes(n.z, n.w), odd_bytes(n.z, n.w));
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          part = dp4a((wv[2 * q] << 4) & 0xF0F0F0F0u, xe[q].x, part);  // 16 q, even k
+          part = dp4a(wv[2 * q] & 0xF0F0F0F0u, xe[q].y, part);         // 16 q, odd k
+          part = dp4a((wv[2 * q + 1] << 4) & 0xF0F0F0F0u, xe[q].z, part);
+          part = dp4a(wv[2 * q + 1] & 0xF0F0F0F0u, xe[q].w, part);
+        }
       } else {
-        part = dp4a_ss((int)w0, (int)xv.x, 0);
-        part = dp4a_ss((int)w1, (int)xv.y, part);
-        part = dp4a_ss((int)w2, (int)xv.z, part);
-        part = dp4a_ss((int)w3, (int)xv.w, part);
+        const uint4* xp = reinterpret_cast<const uint4*>(xs + (size_t)m * K + xoff);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 xv = FUSED ? xp[q] : __ldg(xp + q);
+          part = dp4a(pc.v[q].x, xv.x, part);
+          part = dp4a(pc.v[q].y, xv.y, part);
+          part = dp4a(pc.v[q].z, xv.z, part);
+          part = dp4a(pc.v[q].w, xv.w, part);
+        }
       }
-      if (a.P != nullptr) {
-        int v = part;
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        if (c == 0) a.P[((size_t)m * p.N + row) * C + j] = v;
+      if constexpr (DEBUG) {
+        int v = part + __shfl_xor_sync(0xffffffffu, part, 1);
+        if (h == 0) a.P[((size_t)m * p.N + row) * C + j] = is4 ? (v >> 4) : v;
       }
       acc[m] = fmaf(small_int_to_float(part), sw, acc[m]);
     }
-    if (t == 0 && issued < C) {  // refill stage s once every warp has read it
-      if (!mbar_wait(&empty[s], ph, abort_flag)) {
-        *abort_flag = 1;
-        record_error(a.ws, AQ_ERR_TIMEOUT, 21);
-        ok = false;
-        break;
+  };
+
+  for (int i0 = 0; i0 < nmine; i0 += kRing) {
+#pragma unroll
+    for (int q = 0; q < kRing; ++q) {
+      const int i = i0 + q;
+      if (i < nmine) {
+        tile(i, ring[q]);
+        if (i + kRing < nmine) load(i + kRing, ring[q]);  // read kRing tiles from now
       }
-      issue(issued++);
     }
   }
-  if (t == 0 && !ok) {
-    // let every issued copy land before the CTA's shared memory is released
-    for (int jj = (issued > NS ? issued - NS : 0); jj < issued; ++jj)
-      mbar_wait(&full[jj % NS], (uint32_t)(jj / NS) & 1u, never_flag);
-  }
-  if (!ok || a.P != nullptr) return;
+  if constexpr (DEBUG) return;
 
-  const float bias = p.bias ? __ldg(p.bias + row) : 0.f;
+  // combine the 2 lanes of a row, then the KG groups, in a fixed order
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     if (m >= M) break;
-    float v = acc[m];
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    if (c == 0) store_out(p.y, a.ydtype, (size_t)m * p.ldy + row, fmaf(sxp[m], v, bias));
+    const float v = acc[m] + __shfl_xor_sync(0xffffffffu, acc[m], 1);
+    if (h == 0) red[kg][lrow][m] = v;
+  }
+  __syncthreads();
+  if (kg == 0 && h == 0) {
+    const float bias = p.bias ? __ldg(p.bias + row) : 0.f;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m >= M) break;
+      float v = red[0][lrow][m];
+      for (int q = 1; q < KG; ++q) v += red[q][lrow][m];
+      store_out(p.y, a.ydtype, (size_t)m * p.ldy + row, fmaf(sxp[m], v, bias));
+    }
   }
 }
 
-template <int MT, bool FUSED>
+template <int MT, bool FUSED, bool DEBUG>
 cudaError_t launch_rows_t(const RowsArgs& a, int blocks, size_t smem, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(decode_rows_kernel<MT, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(kMaxStages * kStageBytes + kFusedMaxBytes));
+    cudaError_t e = cudaFuncSetAttribute(decode_rows_kernel<MT, FUSED, DEBUG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedMaxBytes);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_pdl(decode_rows_kernel<MT, FUSED>, dim3(blocks), dim3(kThreads), smem, st, a);
+  return launch_pdl(decode_rows_kernel<MT, FUSED, DEBUG>, dim3(blocks), dim3(kGroupThreads * a.KG), smem, st, a);
 }
 
-template <bool FUSED>
+template <bool FUSED, bool DEBUG>
 cudaError_t launch_rows_m(const RowsArgs& a, int blocks, size_t smem, cudaStream_t st) {
-  if (a.M <= 1) return launch_rows_t<1, FUSED>(a, blocks, smem, st);
-  if (a.M <= 2) return launch_rows_t<2, FUSED>(a, blocks, smem, st);
-  if (a.M <= 4) return launch_rows_t<4, FUSED>(a, blocks, smem, st);
-  return launch_rows_t<8, FUSED>(a, blocks, smem, st);
+  if (a.M <= 1) return launch_rows_t<1, FUSED, DEBUG>(a, blocks, smem, st);
+  if (a.M <= 2) return launch_rows_t<2, FUSED, DEBUG>(a, blocks, smem, st);
+  if (a.M <= 4) return launch_rows_t<4, FUSED, DEBUG>(a, blocks, smem, st);
+  return launch_rows_t<8, FUSED, DEBUG>(a, blocks, smem, st);
 }
 
 }  // namespace
 
 bool rows_supported(int M, int K) { return M >= 1 && M <= kRowsMaxM && K / kTileK <= kMaxC; }
 
-bool rows_fusable(int M, int K) { return (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
+bool rows_fusable(int M, int K) { return 2 * (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
 
 cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
-                               const float* sx, int M, int ydtype, int32_t* P, void* ws, cudaStream_t st) {
+                               const float* sx, int M, int ydtype, int32_t* P, void* /*ws*/, cudaStream_t st) {
   RowsArgs a;
   memset(&a, 0, sizeof(a));
   int blocks = 0;
@@ -307,11 +343,15 @@ cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint
     blocks += a.p[g].blocks;
   }
   a.G = G; a.K = K; a.C = K / kTileK; a.M = M; a.ydtype = ydtype;
-  a.NS = a.C < kMaxStages ? a.C : kMaxStages;
-  a.x = x; a.ldx = ldx; a.xq = xq; a.sx = sx; a.P = P; a.ws = ws;
-  const size_t ring = (size_t)a.NS * kStageBytes;
-  if (x != nullptr) return launch_rows_m<true>(a, blocks, ring + (size_t)M * K + 16 * (size_t)M, st);
-  return launch_rows_m<false>(a, blocks, ring, st);
+  a.x = x; a.ldx = ldx; a.xq = xq; a.sx = sx; a.P = P;
+  // split the tile columns of a CTA over KG thread groups so that ~16 warps per SM stay busy
+  const int warps = blocks * (kGroupThreads / 32);
+  int KG = 1;
+  while (KG < kMaxKG && warps * KG < 16 * kNumSMs && a.C >= 4 * KG) KG *= 2;
+  a.KG = KG;
+  if (P != nullptr) return launch_rows_m<false, true>(a, blocks, 0, st);
+  if (x != nullptr) return launch_rows_m<true, false>(a, blocks, 2 * (size_t)M * K + 16 * (size_t)M, st);
+  return launch_rows_m<false, false>(a, blocks, 0, st);
 }
 
 }  // namespace aq

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __r
   for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, red[w]);
 
   const double s = act_scale(amax);
-  const float r32 = static_cast<float>(1.0 / s);
+  const float r32 = act_recip(s);
   if (threadIdx.x == 0) sx[m] = static_cast<float>(s);
 
 #pragma unroll

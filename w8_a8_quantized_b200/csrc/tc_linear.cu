@@ -124,7 +124,9 @@ __device__ __forceinline__ void store_y(void* y, int ydtype, size_t idx, float v
     reinterpret_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
 }
 
-template <int NT>
+// MODE: 0 = outputs written directly (one split), 1 = split-K partial sums
+// reduced by the last CTA of each unit group, 2 = exact tile products only.
+template <int NT, int MODE>
 __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
     tc_linear_kernel(const __grid_constant__ CUtensorMap tm_w8, const __grid_constant__ CUtensorMap tm_w4,
                      const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
@@ -331,14 +333,23 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
       float acc[kCols];
 #pragma unroll
       for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
+      // tile scale and kind of the next input tile are loaded one tile ahead
+      auto load_scale = [&](int j, uint32_t& swb, uint32_t& lab) {
+        if (rvalid) {
+          const int tt = r * a.C + j;
+          swb = __ldg(a.scales + (size_t)tt * a.bN + nl);
+          lab = __ldg(a.bitmap + (tt >> 3)) >> (tt & 7);
+        }
+      };
+      uint32_t swb_next = 0, lab_next = 0;
+      load_scale(x.j0, swb_next, lab_next);
       for (int j = x.j0; j < x.j1; ++j, ++kt) {
         const int ab = kt & 1;
-        const int tt = r * a.C + j;
+        const uint32_t swb = swb_next, lab = lab_next;
+        if (j + 1 < x.j1) load_scale(j + 1, swb_next, lab_next);
         // INT4 tiles were multiplied by 16 during expansion
-        const bool t4 = rvalid && ((__ldg(a.bitmap + (tt >> 3)) >> (tt & 7)) & 1);
-        const float sw = rvalid ? __half2float(__ushort_as_half(__ldg(a.scales + (size_t)tt * a.bN + nl))) *
-                                      (t4 ? 0.0625f : 1.0f)
-                                : 0.f;
+        const bool t4 = rvalid && (lab & 1);
+        const float sw = rvalid ? __half2float(__ushort_as_half((unsigned short)swb)) * (t4 ? 0.0625f : 1.0f) : 0.f;
         // warp-uniform outcome: the tensor-memory loads below are warp-collective
         if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[ab], (kt >> 1) & 1, abort_flag))) {
           fail(6);
@@ -353,7 +364,7 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
           tmem_ld16(taddr + c16 * 16, v);
           tmem_wait_ld();
           tmem_st16_const(taddr + c16 * 16, kAccBias);  // re-bias for the buffer's next use
-          if (a.P != nullptr) {
+          if constexpr (MODE == 2) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int m = mcol0 + c16 * 16 + i;
@@ -372,8 +383,8 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&tmem_empty[ab]);
       }
-      if (!ok || a.P != nullptr) continue;
-      if (a.S == 1) {
+      if (!ok || MODE == 2) continue;
+      if constexpr (MODE == 0) {
         if (rvalid) {
           const float b = a.bias ? __ldg(a.bias + n) : 0.f;
 #pragma unroll
@@ -457,12 +468,12 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT>
+template <int NT, int MODE>
 cudaError_t launch_nt(const aq_packed* w, const int8_t* xq, TcArgs a, int grid, cudaStream_t st) {
   using Sh = TcShape<NT>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_linear_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_linear_kernel<NT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Sh::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -475,7 +486,7 @@ cudaError_t launch_nt(const aq_packed* w, const int8_t* xq, TcArgs a, int grid, 
   if (w->T4 > 0 && !make_map(&m4, w->w4, kTileK / 2, (uint64_t)w->T4 * w->bN, kTileK / 2, w->bN, false))
     return cudaErrorInvalidValue;
   if (!make_map(&mx, xq, w->K, a.M, kTileK, NT, true)) return cudaErrorInvalidValue;
-  return launch_pdl(tc_linear_kernel<NT>, dim3(grid), dim3(Sh::kThreads), (size_t)Sh::kSmemBytes, st, m8, m4, mx, a);
+  return launch_pdl(tc_linear_kernel<NT, MODE>, dim3(grid), dim3(Sh::kThreads), (size_t)Sh::kSmemBytes, st, m8, m4, mx, a);
 }
 
 }  // namespace
@@ -511,13 +522,21 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
   }
   a.units = a.nrb * a.ntb * a.S;
   const int grid = std::min(a.units, kNumSMs);
-  switch (nt) {
-    case 16: return launch_nt<16>(w, xq, a, grid, st);
-    case 32: return launch_nt<32>(w, xq, a, grid, st);
-    case 48: return launch_nt<48>(w, xq, a, grid, st);
-    case 64: return launch_nt<64>(w, xq, a, grid, st);
-    case 128: return launch_nt<128>(w, xq, a, grid, st);
-    default: return launch_nt<256>(w, xq, a, grid, st);
+  const int mode = P ? 2 : (a.S > 1 ? 1 : 0);
+  switch (nt * 4 + mode) {
+#define AQ_TC_CASE(NTV)                                                  \
+  case NTV * 4 + 0: return launch_nt<NTV, 0>(w, xq, a, grid, st);      \
+  case NTV * 4 + 1: return launch_nt<NTV, 1>(w, xq, a, grid, st);      \
+  case NTV * 4 + 2: return launch_nt<NTV, 2>(w, xq, a, grid, st);
+    AQ_TC_CASE(16)
+    AQ_TC_CASE(32)
+    AQ_TC_CASE(48)
+    AQ_TC_CASE(64)
+    AQ_TC_CASE(128)
+    case 256 * 4 + 0: return launch_nt<256, 0>(w, xq, a, grid, st);
+    case 256 * 4 + 2: return launch_nt<256, 2>(w, xq, a, grid, st);
+#undef AQ_TC_CASE
+    default: return cudaErrorInvalidValue;
   }
 }
 
