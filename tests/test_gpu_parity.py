@@ -245,3 +245,20 @@ def test_group_rejects_mismatched_inputs():
         aq.Group([ws[0], w2], aq.AQ_PHASE_DECODE, 4)
     with pytest.raises(ValueError):
         aq.Group(ws, aq.AQ_PHASE_DECODE, 65)
+
+
+def test_quant_act_every_bf16_absmax():
+    """Every positive finite bf16 value as a row's absmax: the scale (and the codes)
+    must match the oracle's fp64 division bit for bit."""
+    amax_bits = np.arange(1, 0x7F80, dtype=np.uint32).astype(np.uint16)
+    x = np.zeros((amax_bits.size, 16), np.uint16)
+    x[:, 0] = amax_bits
+    x[:, 1] = amax_bits | 0x8000                                   # -amax
+    x[:, 2:] = synth.activations(amax_bits.size, 14, (77,))         # small values
+    xv = oracle.bf16_bits_to_f64(x).astype(np.float32)
+    xv[:, 2:] = np.minimum(np.abs(xv[:, 2:]), oracle.bf16_bits_to_f64(amax_bits)[:, None].astype(np.float32)) * np.sign(xv[:, 2:])
+    x = synth.f32_to_bf16_bits(xv)
+    xq, sx = aq.aq_quant_act(dev_bf16(x))
+    xq_ref, sx_ref = oracle.quant_act(x)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), sx_ref.view(np.uint32))
+    assert np.array_equal(xq.cpu().numpy(), xq_ref)

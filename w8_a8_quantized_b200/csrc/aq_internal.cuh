@@ -264,42 +264,64 @@ __device__ __forceinline__ float abs_max8(const uint4& v, float m) {
   return m;
 }
 
-// s = max(amax / 127, 1e-12) in fp64 (eq. 6 floor).
+// s = max(fl64(amax / 127), 1e-12) (eq. 6 floor).  The quotient is formed from
+// the rounded reciprocal R = fl64(1/127) and one exact residual correction:
+// q = amax R, r = fma(-q, 127, amax) (exact), s = fma(r, R, q).  For every
+// finite bf16 amax this equals the IEEE fp64 quotient (checked exhaustively),
+// at a fraction of a division's latency.
 __device__ __forceinline__ double act_scale(float amax) {
-  double s = static_cast<double>(amax) / 127.0;
+  constexpr double kInv127 = 1.0 / 127.0;
+  const double a = static_cast<double>(amax);
+  const double q = a * kInv127;
+  double s = fma(fma(-q, 127.0, a), kInv127, q);
   return s < 1e-12 ? 1e-12 : s;
 }
 
 // r32 for quant_code: fp32 reciprocal of fp32(s), relative error <= 2 * 2^-24.
 __device__ __forceinline__ float act_recip(double s) { return __frcp_rn(static_cast<float>(s)); }
 
-// clamp(rint(x / s), -127, 127) with x / s rounded in fp64, as the oracle does.
-// Fast path: t = x * r32 carries at most three roundings of 2^-24 each
-// (fp32(s), the reciprocal, the product), so |t - x/s| <= 127 * 3 * 2^-24
-// < 2.3e-5 (|x / s| <= 127).  When t is more than 4e-5 away from the nearest
-// half-integer the exact quotient, and its fp64 rounding, round to the same
-// integer as t; otherwise (ties and near-ties) the fp64 division decides.
-__device__ __forceinline__ int quant_code(float x, double s, float r32) {
-  const float t = x * r32;
-  const float k = rintf(t);
-  if (0.5f - fabsf(t - k) > 4.0e-5f) return static_cast<int>(fminf(fmaxf(k, -127.f), 127.f));
+// clamp(rint(fl64(x / s)), -127, 127): the oracle's rule, by fp64 division.
+static __device__ __noinline__ int quant_code_exact(float x, double s) {
   const double q = rint(static_cast<double>(x) / s);
   return static_cast<int>(fmin(fmax(q, -127.0), 127.0));
 }
 
+// Eight codes of clamp(rint(fl64(x / s)), -127, 127).
+// Fast path: t = x * r32 carries at most three roundings of 2^-24 each
+// (fp32(s), the reciprocal, the product), so |t - x/s| <= 127 * 3 * 2^-24
+// < 2.3e-5 (|x / s| <= 127).  When t is more than 4e-5 away from the nearest
+// half-integer the exact quotient, and its fp64 rounding, round to the same
+// integer as t.  Ties and near-ties (rare) are redone by fp64 division; the
+// warp votes so that the division is a real branch, never paid by every element.
 __device__ __forceinline__ uint2 quantize8(const uint4& v, double s, float r32) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float xf[8];
+  int code[8];
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    xf[i] = bf16_bits_to_float((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
+    const float t = xf[i] * r32;
+    const float k = rintf(t);
+    slow |= !(0.5f - fabsf(t - k) > 4.0e-5f);
+    code[i] = static_cast<int>(fminf(fmaxf(k, -127.f), 127.f));
+  }
+  if (__any_sync(__activemask(), slow)) {
+    if (slow) {
+#pragma unroll 1
+      for (int i = 0; i < 8; ++i) code[i] = quant_code_exact(xf[i], s);
+    }
+  }
   uint32_t out[2];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int c0 = quant_code(bf16_bits_to_float(w[2 * h] & 0xFFFFu), s, r32);
-    const int c1 = quant_code(bf16_bits_to_float(w[2 * h] >> 16), s, r32);
-    const int c2 = quant_code(bf16_bits_to_float(w[2 * h + 1] & 0xFFFFu), s, r32);
-    const int c3 = quant_code(bf16_bits_to_float(w[2 * h + 1] >> 16), s, r32);
-    out[h] = (uint32_t)(c0 & 0xFF) | ((uint32_t)(c1 & 0xFF) << 8) | ((uint32_t)(c2 & 0xFF) << 16) |
-             ((uint32_t)(c3 & 0xFF) << 24);
-  }
+  for (int h = 0; h < 2; ++h)
+    out[h] = (uint32_t)(code[4 * h] & 0xFF) | ((uint32_t)(code[4 * h + 1] & 0xFF) << 8) |
+             ((uint32_t)(code[4 * h + 2] & 0xFF) << 16) | ((uint32_t)(code[4 * h + 3] & 0xFF) << 24);
   return make_uint2(out[0], out[1]);
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }
 
 #endif  // __CUDACC__

@@ -11,7 +11,9 @@
 // Work split: one CTA owns kRows = 32 consecutive output rows of one
 // projection and ALL of its input tiles, so there is no cross-CTA reduction.
 // The CTA has KG groups of 64 threads (KG = 1..8, chosen so the launch keeps
-// about 16 warps per SM busy); group kg takes tile columns kg, kg + KG, ...
+// about 16 warps per SM busy; at most 256 threads for short rows so that the
+// CTAs of the next launch fit beside it and programmatic dependent launch can
+// overlap them); group kg takes tile columns kg, kg + KG, ...
 // In a group, thread t owns row t / 2 and half h = t % 2 of every tile row:
 // input columns [64h, 64h + 64), i.e. 64 contiguous bytes of an INT8 tile row
 // (four 16-byte loads) or 32 bytes of an INT4 tile row (two).  A warp reads 16
@@ -109,20 +111,46 @@ __global__ void __launch_bounds__(kMaxThreads) decode_rows_kernel(const __grid_c
   const int row = row0 + lrow;
   const int tile0 = r * C;
 
-  // ---- per-CTA tile table and scales (independent of earlier kernels)
-  for (int w = t; w < (C + 31) / 32; w += nthr) tile_is4[w] = 0u;
-  __syncthreads();
-  for (int j = t; j < C; j += nthr) {
-    const int tt = tile0 + j;
-    const int is4 = (__ldg(p.bitmap + (tt >> 3)) >> (tt & 7)) & 1;
-    const size_t pr = (size_t)__ldg(p.tile_idx + tt) * bN + nl0;
-    tile_ptr[j] = is4 ? p.w4 + pr * (kTileK / 2) : reinterpret_cast<const uint8_t*>(p.w8) + pr * kTileK;
-    if (is4) atomicOr(&tile_is4[j >> 5], 1u << (j & 31));
-  }
-  for (int q = t; q < 4 * C; q += nthr) {  // 32 rows x 2 B = four 16-byte pieces per tile column
-    const int j = q >> 2, part = q & 3;
-    *reinterpret_cast<uint4*>(&tile_sw[j][8 * part]) =
-        __ldg(reinterpret_cast<const uint4*>(p.scales + (size_t)(tile0 + j) * bN + nl0 + 8 * part));
+  // ---- per-CTA tile table and scales (independent of earlier kernels): the loads
+  // of a pass are all issued before any is used (one round trip for C <= 2 nthr)
+  for (int base = 0; base < C; base += 2 * nthr) {
+    int idx[2];
+    uint32_t lab[2];
+    uint4 scv[8];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int j = base + t + q * nthr;
+      if (j < C) {
+        const int tt = tile0 + j;
+        lab[q] = __ldg(p.bitmap + (tt >> 3)) >> (tt & 7);
+        idx[q] = __ldg(p.tile_idx + tt);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {  // 32 rows x 2 B = four 16-byte pieces per tile column
+      const int e = 4 * base + t + q * nthr;
+      if (e < 4 * C)
+        scv[q] = __ldg(reinterpret_cast<const uint4*>(p.scales + (size_t)(tile0 + (e >> 2)) * bN + nl0 + 8 * (e & 3)));
+    }
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int j0 = base + q * nthr + (t & ~31);  // first tile column of this warp's label word
+      if (j0 < C) {
+        const int j = base + t + q * nthr;
+        const bool is4 = j < C && (lab[q] & 1);
+        const unsigned bits = __ballot_sync(0xffffffffu, is4);
+        if (lane == 0) tile_is4[j0 >> 5] = bits;
+        if (j < C) {
+          const size_t pr = (size_t)idx[q] * bN + nl0;
+          tile_ptr[j] = is4 ? p.w4 + pr * (kTileK / 2) : reinterpret_cast<const uint8_t*>(p.w8) + pr * kTileK;
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = 4 * base + t + q * nthr;
+      if (e < 4 * C) *reinterpret_cast<uint4*>(&tile_sw[e >> 2][8 * (e & 3)]) = scv[q];
+    }
   }
   __syncthreads();
   pdl_launch_dependents();
@@ -147,6 +175,12 @@ __global__ void __launch_bounds__(kMaxThreads) decode_rows_kernel(const __grid_c
 #pragma unroll
   for (int q = 0; q < kRing; ++q)
     if (q < nmine) load(q, ring[q]);
+  if constexpr (FUSED) {
+    // warm L2 with the activations: L2 is coherent, so this is safe even if an
+    // earlier kernel is still writing them (the reads below come after the wait)
+    const int nlines = (M * a.ldx * 2 + 127) / 128;
+    for (int q = t; q < nlines; q += nthr) prefetch_l2(reinterpret_cast<const uint8_t*>(a.x) + 128 * (size_t)q);
+  }
 
   pdl_wait();  // activations (and every global write below) depend on earlier kernels
 
@@ -346,8 +380,10 @@ cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint
   a.x = x; a.ldx = ldx; a.xq = xq; a.sx = sx; a.P = P;
   // split the tile columns of a CTA over KG thread groups so that ~16 warps per SM stay busy
   const int warps = blocks * (kGroupThreads / 32);
+  // at most 256 threads (room for the next launch's CTAs) unless rows are long
+  const int kg_cap = a.C >= 32 ? kMaxKG : 4;
   int KG = 1;
-  while (KG < kMaxKG && warps * KG < 16 * kNumSMs && a.C >= 4 * KG) KG *= 2;
+  while (KG < kg_cap && warps * KG < 16 * kNumSMs && a.C >= 4 * KG) KG *= 2;
   a.KG = KG;
   if (P != nullptr) return launch_rows_m<false, true>(a, blocks, 0, st);
   if (x != nullptr) return launch_rows_m<true, false>(a, blocks, 2 * (size_t)M * K + 16 * (size_t)M, st);
