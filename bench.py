@@ -54,6 +54,31 @@ WORKLOADS = {
     "prefill-qwen3-14b": dict(model="qwen3-14b", phase="prefill", bN=128, frac8=0.30, M=8192, extra_M=(),
                               outlier=0.01),
 }
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels,
+# from the ncu captures summarised in profiles/, valid only while the kernel source is unchanged
+# (sha256 prefix of the source file and the shared header).
+MEASURED_TRAFFIC = {
+    # profiles/decode_rows_llama3b_1token.md: one layer's four launches read 64,728,320 B and wrote
+    # 5,120 B -> 16,183,360 B per launch (algorithmic: 16,128,638 B per launch)
+    "decode": {"src": ("w8_a8_quantized_b200/csrc/decode_rows.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
+               "sha": "75c2b2e21933c4bb", "bytes_per_launch": 16183360},
+    "prefill": {"src": ("w8_a8_quantized_b200/csrc/tc_linear.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
+                "sha": None, "bytes_per_launch": None},
+}
+
+
+def measured_traffic(phase: str):
+    import hashlib
+    rec = MEASURED_TRAFFIC[phase]
+    if rec["sha"] is None:
+        return None
+    h = hashlib.sha256()
+    for f in rec["src"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return rec["bytes_per_launch"] if h.hexdigest()[:16] == rec["sha"] else None
+
+
 CFG_ID = {"llama-3.2-3b": 2, "qwen3-4b": 3, "dense-8b": 4, "qwen3-14b": 5, "single-2048": 1}
 INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out", "gate": "mlp_in", "up": "mlp_in",
             "down": "mlp_hidden"}
@@ -85,7 +110,7 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling (200 ms) of SM clock and throttle reasons while running."""
+    """nvidia-smi sampling (every 50 ms) of SM clock and throttle reasons while running."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -98,7 +123,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -415,7 +440,8 @@ def main():
         value = world * wbytes / (r0["ms"] * 1e-3) / 1e9
         achieved = wbytes / (r0["ms_linear_only"] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm"], "traffic": None,
+                "frac": achieved / peaks["hbm"], "traffic": measured_traffic("decode"),
+                "algorithmic_bytes_per_launch": wbytes / r0["linear_launches"],
                 "kernel": "decode linear (all projections, activation quantization excluded)",
                 "peak_source": peaks["src"]}
         e2e_val = world * wbytes / (r0["ms_e2e"] * 1e-3) / 1e9
@@ -426,7 +452,7 @@ def main():
         achieved = ops / (r0["ms_linear_only"] * 1e-3) / 1e12
         int8_peak = 2.0 * peaks["bf16"]  # dense INT8 = 2x dense BF16 (nominal ratio 4.5 / 2.25)
         roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
-                "frac": achieved / int8_peak, "traffic": None,
+                "frac": achieved / int8_peak, "traffic": measured_traffic("prefill"),
                 "kernel": "prefill linear (all projections, activation quantization excluded)",
                 "peak_source": f"{peaks['src']} bf16 x 2"}
         e2e_val = world * ops / (r0["ms_e2e"] * 1e-3) / 1e12
