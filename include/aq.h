@@ -214,6 +214,33 @@ int aq_linear_group(int phase, const aq_packed* const* w, int G, const uint16_t*
 size_t aq_group_workspace_bytes(int phase, int M, const aq_packed* const* w, int G);
 
 /*
+ * Decode-phase linear layer for callers that cannot allocate device memory
+ * (code running inside an allocator or memory-pool callback, runtimes that
+ * forbid allocation after start-up to keep a fixed footprint, plug-ins handed
+ * only their input and output buffers).  The paper has no counterpart: this is
+ * a deployment convenience of this library.
+ *
+ * Same arguments and result as aq_linear_decode, without the workspace: the
+ * split-K scratch comes from a fixed 4 MiB array in device memory that the
+ * library holds on every GPU that loads it, until the process exits.
+ *  - Allocates nothing and calls no allocating routine.
+ *  - The first call on a device resolves the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture on the device.
+ *  - Each call clears the parts of the array that must start at zero (status
+ *    word, split-K counters) on `stream` before launching.
+ *  - All calls share the one array: calls that overlap on the GPU (different
+ *    streams, or graphs replayed concurrently) race and produce wrong results.
+ *  - A call whose scratch need (aq_workspace_bytes(AQ_PHASE_DECODE, M, w))
+ *    exceeds 4 MiB is rejected with AQ_ERR_WORKSPACE; use aq_linear_decode.
+ *  - No status query exists for this array; a bounded wait that gives up
+ *    inside the kernel leaves y unspecified.
+ * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ */
+int aq_linear_decode_noalloc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                             void* y, int ydtype, int ldy, void* stream);
+
+/*
  * Synchronizes `stream`, then reads and clears the error word a kernel left in
  * the workspace `ws`.  Returns AQ_OK, AQ_ERR_TIMEOUT (a bounded wait inside a
  * kernel gave up; *info, nullable, receives where) or AQ_ERR_CUDA.

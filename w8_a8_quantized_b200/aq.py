@@ -21,7 +21,7 @@ AQ_PHASE_DECODE, AQ_PHASE_PREFILL = 0, 1
 BUF_NAMES = ("bitmap", "row_off4", "row_off8", "tile_idx", "w4", "w8", "scales")
 EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "aq_quant_act",
             "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
-            "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status")
+            "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc")
 
 
 class AqError(RuntimeError):
@@ -74,6 +74,8 @@ def lib():
                                   c_void_p]
     L.aq_group_workspace_bytes.restype = c_size_t
     L.aq_group_workspace_bytes.argtypes = [c_int, c_int, ctypes.POINTER(P), c_int]
+    L.aq_linear_decode_noalloc.restype = c_int
+    L.aq_linear_decode_noalloc.argtypes = [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p]
     L.aq_workspace_status.restype = c_int
     L.aq_workspace_status.argtypes = [c_void_p, c_void_p, ctypes.POINTER(c_int)]
     _lib = L
@@ -215,6 +217,27 @@ def aq_linear_prefill(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=t
     """Prefill-phase y (tensor-core INT8 path), any M >= 1."""
     return _linear(lib().aq_linear_prefill, "aq_linear_prefill", AQ_PHASE_PREFILL, w, xq, sx, bias, out, out_dtype,
                    ws)
+
+
+def aq_linear_decode_noalloc(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=torch.float32):
+    """aq_linear_decode without a workspace, for callers that cannot allocate device
+    memory: the library's fixed 4 MiB device scratch is used instead (calls that
+    overlap on the GPU must not share it).  `out` must be preallocated by callers
+    that cannot allocate; it is allocated here only for convenience."""
+    _need(xq, "xq", torch.int8, w.device)
+    _need(sx, "sx", torch.float32, w.device)
+    M = xq.shape[0]
+    if out is None:
+        out = torch.empty((M, w.N), dtype=out_dtype, device=w.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or out.stride(1) != 1 or out.device != w.device:
+        raise ValueError("out must be float32 or bfloat16 on the weights' device with unit inner stride")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, w.device)
+    _check(lib().aq_linear_decode_noalloc(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
+                                          bias.data_ptr() if bias is not None else None, out.data_ptr(),
+                                          AQ_F32 if out.dtype == torch.float32 else AQ_BF16, out.stride(0),
+                                          _stream(w.device)), "aq_linear_decode_noalloc")
+    return out
 
 
 class Group:

@@ -53,6 +53,7 @@ struct DecodeProj {
   void* y;
   int N, bN, ldy, blocks;
 };
+DecodeProj decode_proj(const aq_packed* w, const float* bias, void* y, int ldy);
 bool rows_supported(int M, int K);
 bool rows_fusable(int M, int K);
 cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
