@@ -72,7 +72,9 @@ typedef enum { AQ_PHASE_DECODE = 0, AQ_PHASE_PREFILL = 1 } aq_phase;
  *                                  as uint16, logical tile order
  *
  * Inside a tile both precisions use the same element order: output row, then
- * input column.
+ * input column.  w4, w8 and scales must start on a 16-byte boundary (the
+ * kernels move them with bulk copies); a packed layout that breaks this is
+ * rejected with AQ_ERR_ARG.
  */
 typedef struct aq_packed {
   int32_t N, K, bN, bK, R, C, T4, T8;

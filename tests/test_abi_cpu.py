@@ -113,6 +113,11 @@ def test_host_validation_rejects_before_any_launch():
     assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 64, 16, 1 << 20, None) == -1
     assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, None, 0, None) == -5
     assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, 16, 8, None) == -5
+    # packed buffers moved by bulk copies (w4, w8, scales) must be 16-byte aligned
+    mis = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
+                            bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=18)
+    assert L.aq_linear_prefill(ctypes.byref(mis), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_decode(ctypes.byref(mis), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
     assert L.aq_workspace_bytes(0, 65, ctypes.byref(s)) == 0
     assert L.aq_workspace_bytes(0, 1, ctypes.byref(s)) >= 256
     assert L.aq_workspace_bytes(5, 1, ctypes.byref(s)) == 0

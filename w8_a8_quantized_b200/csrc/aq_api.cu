@@ -15,7 +15,7 @@ int validate_packed(const aq_packed* w) {
   if (w->T4 < 0 || w->T8 < 0 || (long long)w->T4 + w->T8 != (long long)w->R * w->C) return AQ_ERR_SHAPE;
   if (!w->bitmap || !w->row_off4 || !w->row_off8 || !w->tile_idx || !w->scales) return AQ_ERR_ARG;
   if ((w->T4 > 0 && !w->w4) || (w->T8 > 0 && !w->w8)) return AQ_ERR_ARG;
-  if (((uintptr_t)w->w4 & 15) || ((uintptr_t)w->w8 & 15)) return AQ_ERR_ARG;
+  if (((uintptr_t)w->w4 & 15) || ((uintptr_t)w->w8 & 15) || ((uintptr_t)w->scales & 15)) return AQ_ERR_ARG;
   return AQ_OK;
 }
 

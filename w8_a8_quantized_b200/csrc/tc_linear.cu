@@ -6,28 +6,55 @@
 // an exact INT32 sum, and each is rescaled by its activation and weight
 // scales before FP32 accumulation over the input tiles.
 //
-// Roles in one CTA (persistent over work units):
-//   warp 0      TMA producer: INT8 tiles -> swizzled A stage, INT4 tiles ->
-//               staging buffer, activation tile -> B stage.
+// Roles in one CTA (persistent over work units; every role walks the same
+// sequence of input tiles g = 0, 1, 2, ... of the CTA's units):
+//   warp 0      weight producer: INT8 tiles -> swizzled A stage (TMA), INT4
+//               tiles -> staging buffer (TMA).  It does not wait for the
+//               previous kernel, so the first stages load while it finishes.
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma
 //               (kind::i8, M = 128 weight rows, N = NT tokens, K = 32) four
-//               times per 128-wide input tile into a double-buffered INT32
-//               accumulator in tensor memory.
-//   warps 2-3   expand INT4 staging tiles into the 128-byte-swizzled INT8
-//               A layout (fence.proxy.async before signalling the MMA).
-//   warps 4..   epilogue: after every input tile, read the INT32 tile product
-//               from tensor memory, multiply by the row's fp16 weight scale of
-//               that tile and accumulate in FP32 registers; at the end of a
-//               work unit multiply by the token scale, add bias and store.
+//               times per 128-wide input tile into one of four INT32
+//               accumulator buffers in tensor memory.
+//   warp 2      tile metadata: all 32 lanes read labels and physical tile
+//               indices (AlignQuant, App. E.2 eq. 16) up to 32 tiles ahead and
+//               turn them into ready-made copy records in a shared-memory
+//               ring, so the producers spend a handful of instructions per tile.
+//   warp 3      activation producer: the NT x 128 INT8 activation tile -> B
+//               stage (TMA), after the previous kernel (which writes the
+//               activations) is done; and the tile's fp16 row scales -> scale
+//               ring (bulk copy) for the epilogue.
+//   warps 4..   epilogue; warp w may read tensor-memory lanes 32 (w % 4) ..
+//               32 (w % 4) + 31.  After every input tile it reads the INT32
+//               tile product from tensor memory, multiplies by the row's fp16
+//               weight scale of that tile and accumulates in FP32 registers;
+//               at the end of a work unit it multiplies by the token scale,
+//               adds bias and stores.
+//               The same warps expand the INT4 staging tiles into the
+//               128-byte-swizzled INT8 A layout kExpandAhead tiles ahead of
+//               the tile they rescale (fence.proxy.async before signalling the
+//               MMA): expansion runs on the integer and load/store pipes beside
+//               the FP32 rescale, and no separate expander warps take
+//               registers from the epilogue.
+// A single thread on a busy SM retires roughly one dependent instruction every
+// 10-20 cycles, so the per-tile work of each issuing thread is kept to a few
+// dozen instructions and spread over three threads.
 // Weights are the A operand, so TMEM lane = output row and each epilogue
 // thread applies ONE weight scale per input tile.
+//
+// The FP32 rescale is the co-bottleneck of this design: per input tile and
+// output element it costs one add and one fused multiply-add on the CUDA
+// cores, as many cycles per SM as the INT8 MMA itself; the float2 forms
+// halve the issue slots it takes so tensor-memory and expansion work fit
+// beside it.
 //
 // A work unit is (128-row block of output features, NT-token block, split of
 // the input tiles).  Split partial sums go to the workspace; the CTA that
 // finishes a unit last sums all splits in increasing split order.
 // Every mbarrier wait is bounded (see mbar_wait); a wait that gives up records
-// AQ_ERR_TIMEOUT in the workspace, raises a CTA-wide abort flag, drains the
-// copies and MMAs it issued, and the CTA frees its tensor memory and exits.
+// AQ_ERR_TIMEOUT in the workspace and raises a CTA-wide abort flag; every
+// role then leaves its loop, the copy issuers give their copies in flight a
+// grace period, the MMA lane waits (bounded) for its MMAs, and the CTA frees
+// its tensor memory and exits.
 #include <algorithm>
 #include <cstring>
 
@@ -36,29 +63,55 @@
 namespace aq {
 namespace {
 
+constexpr int kBufs = 4;        // accumulator buffers in tensor memory
+constexpr int kScSlots = 16;    // scale ring slots (>= stages + kBufs: slots are reused without a barrier)
+constexpr int kMetaSlots = 32;  // metadata ring slots (one per lane of the metadata warp)
+constexpr int kFirstEpiWarp = 4;
+// Tiles the epilogue expands ahead of the one it rescales.  At least kBufs,
+// so the MMA (at most kBufs tiles ahead of the epilogue) never waits for an
+// expansion; below stages + kBufs, so the staging copy it waits for never
+// depends on the epilogue's own later progress.
+constexpr int kExpandAhead = kBufs;
+
 template <int NT>
 struct TcShape {
   static constexpr int kA = 128 * kTileK;        // swizzled INT8 weight block
   static constexpr int kStg = 128 * kTileK / 2;  // INT4 staging (row-major, 64 B per row)
   static constexpr int kB = NT * kTileK;         // swizzled INT8 activation block
   static constexpr int kStageBytes = kA + kB + kStg;
-  static constexpr int kStages = NT >= 256 ? 3 : (NT >= 128 ? 4 : 6);
-  static constexpr int kEpiWarps = NT > 64 ? 4 * (NT / 64) : 4;  // 4 warps (one per lane quadrant) per 64 columns
-  static constexpr int kCols = NT / (kEpiWarps / 4);             // accumulator columns per epilogue thread (<= 64)
-  static constexpr int kThreads = 128 + 32 * kEpiWarps;
-  static constexpr int kTmemCols = 2 * NT <= 32 ? 32 : 2 * NT <= 64 ? 64 : 2 * NT <= 128 ? 128 : 2 * NT <= 256 ? 256 : 512;
-  static constexpr int kBufStride = kTmemCols / 2;  // column offset of accumulator buffer 1
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes < 8 ? (200 * 1024) / kStageBytes : 8;
+  static constexpr int kCols = NT <= 64 ? NT : 64;  // accumulator columns per epilogue thread
+  static constexpr int kEpiWarps = 4 * NT / kCols;      // 4 warps (one per lane quadrant) per column group
+  static constexpr int kThreads = 32 * kFirstEpiWarp + 32 * kEpiWarps;
+  // Tensor-memory columns per load wait: all of them up to 48; 64 columns take
+  // two waits, which keeps the loaded values and the accumulators within the
+  // register budget.
+  static constexpr int kLdCols = kCols <= 48 ? kCols : 32;
+  static_assert(kCols % kLdCols == 0 && kLdCols % 16 == 0, "load chunks");
+  // Registers per thread: the register file over the block's warps, counted in
+  // groups of four warps as the hardware allocates them (an explicit cap: the
+  // block-size bound makes the compiler trade registers for spills here).
+  static constexpr int kMaxRegsRaw = 65536 / (128 * ((kThreads + 127) / 128)) / 8 * 8;
+  static constexpr int kMaxRegs = kMaxRegsRaw > 255 ? 255 : kMaxRegsRaw;
+  static constexpr int kTmemCols = kBufs * NT <= 32 ? 32 : kBufs * NT <= 64 ? 64 : kBufs * NT <= 128 ? 128
+                                   : kBufs * NT <= 256 ? 256 : 512;
+  static constexpr int kScBytes = kScSlots * 256;  // 128 rows x fp16 per slot
+  static constexpr int kCtrlBytes = 2048;
+  static constexpr int kPreBytes = (32 + kCols) * kEpiWarps * 4;  // per-unit bias and token scales of the epilogue
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kScBytes + kCtrlBytes + kPreBytes;
   static constexpr uint32_t kIdesc = idesc_i8(128, NT);
-  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N");
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "MMA N");
+  static_assert(kBufs * NT <= 512, "tensor memory");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
-  static_assert((4 * kStages + 5) * 8 + 16 <= kBarBytes, "barrier area");
+  static_assert(kStages >= 3 && kScSlots >= kStages + kBufs, "ring depths");
+  static_assert(kExpandAhead >= kBufs && kExpandAhead < kStages + kBufs, "expansion distance");
+  static_assert(kThreads <= 1024, "block size");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 constexpr uint32_t kAccBias = 0x4B400000u;  // fp32 bit pattern of 12582912 = 1.5 * 2^23
 constexpr float kAccBiasF = 12582912.0f;
+constexpr unsigned long long kAbortGraceNs = 200000;  // copies in flight when a CTA gives up
 
 struct TcArgs {
   const uint8_t* bitmap;
@@ -94,19 +147,64 @@ __device__ __forceinline__ Unit unit_of(const TcArgs& a, int u) {
   return x;
 }
 
-// INT4 label mask (bit sub) and validity mask of the sub-tiles of one input tile.
-__device__ __forceinline__ void tile_kinds(const TcArgs& a, int rb, int j, int& valid, int& is4) {
-  valid = 0;
-  is4 = 0;
-  for (int sub = 0; sub < a.tpb; ++sub) {
-    const int r = rb * a.tpb + sub;
-    if (r < a.R) {
-      valid |= 1 << sub;
-      const int t = r * a.C + j;
-      if ((__ldg(a.bitmap + (t >> 3)) >> (t & 7)) & 1) is4 |= 1 << sub;
+// Walks the CTA's input tiles in the order every role processes them.
+struct TileIter {
+  int u, j;
+  Unit x;
+  __device__ __forceinline__ explicit TileIter(const TcArgs& a) : u(blockIdx.x), j(0) {
+    if (u < a.units) {
+      x = unit_of(a, u);
+      j = x.j0;
+      skip(a);
     }
   }
+  __device__ __forceinline__ void skip(const TcArgs& a) {
+    while (u < a.units && j >= x.j1) {
+      u += gridDim.x;
+      if (u < a.units) {
+        x = unit_of(a, u);
+        j = x.j0;
+      }
+    }
+  }
+  __device__ __forceinline__ void next(const TcArgs& a) {
+    ++j;
+    skip(a);
+  }
+  __device__ __forceinline__ bool valid(const TcArgs& a) const { return u < a.units; }
+};
+
+// Per-tile record of the metadata ring: everything the producers need to
+// issue the tile's copies.
+struct MetaRec {
+  uint32_t a_row0, a_row1;  // first row of each sub-tile's weight tile in its precision's buffer
+  uint32_t sizes;           // INT8 KiB | INT4 KiB << 8 | kinds << 28 (copy sizes are whole KiB)
+  uint32_t sc_off;          // element offset of sub-tile 0's scales (sub-tile 1: + C * bN)
+};
+// kinds: bits 0-1 INT4 label of sub-tile 0/1, bits 2-3 sub-tile 0/1 exists
+// (the last 128-row block of a bN = 64 layer may hold one tile row only).
+
+// Input tiles the CTA processes (identical in every role).
+__device__ __forceinline__ uint32_t cta_tiles(const TcArgs& a) {
+  uint32_t n = 0;
+  for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
+    const Unit x = unit_of(a, u);
+    n += x.j1 - x.j0;
+  }
+  return n;
 }
+
+// Ring position with its phase parity.
+struct RingPos {
+  uint32_t i, ph;
+  template <int N>
+  __device__ __forceinline__ void next() {
+    if (++i == N) {
+      i = 0;
+      ph ^= 1u;
+    }
+  }
+};
 
 // 8 nibbles (low nibble = even k) -> 8 INT8 bytes holding 16 * q in k order.
 // A nibble placed in the high half of a byte with a zero low half IS the
@@ -124,10 +222,33 @@ __device__ __forceinline__ void store_y(void* y, int ydtype, size_t idx, float v
     reinterpret_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
 }
 
+// Orders every later use of r after the preceding tcgen05.wait::ld (the
+// registers written by tcgen05.ld are valid only after that wait).
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+
+// 4-byte global -> shared copy; with src_bytes = 0 it writes zero and reads nothing.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Give bulk / tensor copies already issued time to land before the CTA exits
+// after an abort (their completion can no longer be awaited on a barrier that
+// another role stopped arming).
+__device__ __forceinline__ void abort_grace() {
+  const unsigned long long t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < kAbortGraceNs) __nanosleep(1000);
+}
+
 // MODE: 0 = outputs written directly (one split), 1 = split-K partial sums
 // reduced by the last CTA of each unit group, 2 = exact tile products only.
 template <int NT, int MODE>
-__global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
+__global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
     tc_linear_kernel(const __grid_constant__ CUtensorMap tm_w8, const __grid_constant__ CUtensorMap tm_w4,
                      const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
   using Sh = TcShape<NT>;
@@ -138,32 +259,53 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
   auto stage_a = [&](int st) { return smem + st * Sh::kStageBytes; };
   auto stage_b = [&](int st) { return smem + st * Sh::kStageBytes + Sh::kA; };
   auto stage_g = [&](int st) { return smem + st * Sh::kStageBytes + Sh::kA + Sh::kB; };
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_ * Sh::kStageBytes);
-  uint64_t* full = bars;
-  uint64_t* staged = bars + S_;
-  uint64_t* expanded = bars + 2 * S_;
-  uint64_t* empty = bars + 3 * S_;
-  uint64_t* tmem_full = bars + 4 * S_;
-  uint64_t* tmem_empty = bars + 4 * S_ + 2;
-  uint64_t* epi_sync = bars + 4 * S_ + 4;  // epilogue-only rendezvous (bounded, unlike bar.sync)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4 * S_ + 5);
+  uint8_t* sc_ring = smem + S_ * Sh::kStageBytes;  // [kScSlots][128] fp16
+  uint8_t* ctrl = sc_ring + Sh::kScBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);  // weights (INT8) + activations landed; one arrival per producer
+  uint64_t* staged = full + S_;                        // INT4 staging landed (0 bytes when none)
+  uint64_t* expanded = staged + S_;                    // epilogue warps done expanding the stage (one arrival each)
+  uint64_t* empty = expanded + S_;                     // MMAs reading the stage done
+  uint64_t* tmem_full = empty + S_;
+  uint64_t* tmem_empty = tmem_full + kBufs;
+  uint64_t* sc_full = tmem_empty + kBufs;
+  uint64_t* meta_full = sc_full + kScSlots;
+  uint64_t* meta_empty = meta_full + kMetaSlots;
+  uint64_t* epi_sync = meta_empty + kMetaSlots;  // epilogue-only rendezvous (bounded, unlike bar.sync)
+  uint64_t* drain = epi_sync + 1;                // MMA completion on the way out
+  MetaRec* meta = reinterpret_cast<MetaRec*>(drain + 1);
+  volatile uint32_t* stage_info = reinterpret_cast<volatile uint32_t*>(meta + kMetaSlots);
+  volatile uint32_t* sc_info = stage_info + S_;
+  uint32_t* tmem_slot = const_cast<uint32_t*>(sc_info + kScSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* never_flag = reinterpret_cast<volatile int*>(tmem_slot + 3);  // stays 0: drain waits
+  float* pre_bias = reinterpret_cast<float*>(ctrl + Sh::kCtrlBytes);  // [32 kEpiWarps] bias of each epilogue row
+  float* pre_sx = pre_bias + 32 * Sh::kEpiWarps;                       // [kEpiWarps][kCols] token scales
+  static_assert((4 * 8 + 2 * kBufs + 2 * kScSlots + 2 * kMetaSlots + 2) * 8 + kMetaSlots * 16 + (8 + kScSlots + 4) * 4 <=
+                    Sh::kCtrlBytes,
+                "control area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int st = 0; st < S_; ++st) {
-      mbar_init(&full[st], 1);
+      mbar_init(&full[st], 2);
       mbar_init(&staged[st], 1);
-      mbar_init(&expanded[st], 64);
+      mbar_init(&expanded[st], Sh::kEpiWarps);
       mbar_init(&empty[st], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(&tmem_full[b], 1);
-      mbar_init(&tmem_empty[b], 32 * Sh::kEpiWarps);
+      mbar_init(&tmem_empty[b], Sh::kEpiWarps);
+    }
+    for (int s = 0; s < kScSlots; ++s) {
+      mbar_init(&sc_full[s], 1);
+    }
+    for (int s = 0; s < kMetaSlots; ++s) {
+      mbar_init(&meta_full[s], 1);
+      mbar_init(&meta_empty[s], 2);  // both producers read every record
     }
     mbar_init(epi_sync, 32 * Sh::kEpiWarps);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     *never_flag = 0;
     fence_mbar_init();
@@ -187,187 +329,258 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ weight producer
     if (lane == 0) {
-      pdl_wait();  // activations come from an earlier kernel
-      uint32_t g = 0, stg_bits = 0, stg_used = 0;
+      const uint32_t g_total = cta_tiles(a);
+      RingPos mr{0, 0}, sr{0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
-        const Unit x = unit_of(a, u);
-        for (int j = x.j0; j < x.j1; ++j, ++g) {
-          const int st = g % S_;
-          const uint32_t use = g / S_;
-          if (!mbar_wait(&empty[st], (use & 1) ^ 1, abort_flag)) { fail(1); ok = false; break; }
-          int valid, is4;
-          tile_kinds(a, x.rb, j, valid, is4);
-          uint32_t bytes_full = Sh::kB, bytes_stg = 0;
-          for (int sub = 0; sub < a.tpb; ++sub)
-            if (valid >> sub & 1) {
-              if (is4 >> sub & 1) bytes_stg += a.bN * (kTileK / 2);
-              else bytes_full += a.bN * kTileK;
-            }
-          mbar_arrive_expect_tx(&full[st], bytes_full);
-          if (bytes_stg) {
-            mbar_arrive_expect_tx(&staged[st], bytes_stg);
-            stg_bits ^= 1u << st;
-            stg_used |= 1u << st;
-          }
-          for (int sub = 0; sub < a.tpb; ++sub) {
-            if (!(valid >> sub & 1)) continue;
-            const int t = (x.rb * a.tpb + sub) * a.C + j;
-            const int row = __ldg(a.tile_idx + t) * a.bN;
-            if (is4 >> sub & 1)
-              tma_load_2d(stage_g(st) + sub * a.bN * (kTileK / 2), &tm_w4, 0, row, &staged[st]);
-            else
-              tma_load_2d(stage_a(st) + sub * a.bN * kTileK, &tm_w8, 0, row, &full[st]);
-          }
-          tma_load_2d(stage_b(st), &tm_x, j * kTileK, x.tb * NT, &full[st]);
+      for (uint32_t g = 0; g < g_total; ++g) {
+        if (!mbar_wait(&meta_full[mr.i], mr.ph, abort_flag)) { fail(1); ok = false; break; }
+        const MetaRec rec = meta[mr.i];
+        mbar_arrive(&meta_empty[mr.i]);
+        mr.next<kMetaSlots>();
+        if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(2); ok = false; break; }
+        const uint32_t kinds = rec.sizes >> 28;
+        stage_info[sr.i] = kinds;  // read by the expanding epilogue warps after `staged`
+        mbar_arrive_expect_tx(&full[sr.i], (rec.sizes & 0xFFu) << 10);
+        mbar_arrive_expect_tx(&staged[sr.i], ((rec.sizes >> 8) & 0xFFu) << 10);
+        if (kinds & 1) tma_load_2d(stage_g(sr.i), &tm_w4, 0, rec.a_row0, &staged[sr.i]);
+        else tma_load_2d(stage_a(sr.i), &tm_w8, 0, rec.a_row0, &full[sr.i]);
+        if (kinds & 8) {
+          if (kinds & 2) tma_load_2d(stage_g(sr.i) + a.bN * (kTileK / 2), &tm_w4, 0, rec.a_row1, &staged[sr.i]);
+          else tma_load_2d(stage_a(sr.i) + a.bN * kTileK, &tm_w8, 0, rec.a_row1, &full[sr.i]);
         }
+        sr.next<S_>();
       }
-      if (!ok) {
-        // let every copy already issued land before the CTA's memory goes away
-        for (int st = 0; st < S_ && (uint32_t)st < g; ++st) {
-          const uint32_t last = (g - 1 - st) / S_;  // last use of stage st
-          mbar_wait(&full[st], last & 1, never_flag);
-          if (stg_used >> st & 1) mbar_wait(&staged[st], ((stg_bits >> st) & 1) ^ 1, never_flag);
-        }
-      }
+      if (!ok || *abort_flag) abort_grace();
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t g = 0, kt = 0, exp_bits = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
-        const Unit x = unit_of(a, u);
-        for (int j = x.j0; j < x.j1; ++j, ++g, ++kt) {
-          const int st = g % S_;
-          if (!mbar_wait(&full[st], (g / S_) & 1, abort_flag)) { fail(2); ok = false; break; }
-          int valid, is4;
-          tile_kinds(a, x.rb, j, valid, is4);
-          if (is4) {
-            if (!mbar_wait(&expanded[st], (exp_bits >> st) & 1, abort_flag)) { fail(3); ok = false; break; }
-            exp_bits ^= 1u << st;
-          }
-          const int ab = kt & 1;  // use kt >> 1 of this buffer waits for the epilogue's release number kt >> 1
-          if (!mbar_wait(&tmem_empty[ab], (kt >> 1) & 1, abort_flag)) { fail(4); ok = false; break; }
-          tc_fence_after();
-          const uint64_t adesc = sw128_desc(smem_u32(stage_a(st)));
-          const uint64_t bdesc = sw128_desc(smem_u32(stage_b(st)));
-          const uint32_t d = tmem_base + ab * Sh::kBufStride;
-          // the buffer holds the bias kAccBias in every element; all four MMAs accumulate onto it
+      const uint32_t g_total = cta_tiles(a);
+      const uint64_t adesc0 = sw128_desc(smem_u32(stage_a(0)));
+      const uint64_t bdesc0 = sw128_desc(smem_u32(stage_b(0)));
+      RingPos sr{0, 0}, br{0, 0};
+      uint32_t g = 0;
+      for (; g < g_total; ++g) {
+        if (!mbar_wait(&full[sr.i], sr.ph, abort_flag)) { fail(4); break; }
+        if (!mbar_wait(&expanded[sr.i], sr.ph, abort_flag)) { fail(5); break; }
+        // use u of a buffer waits for the epilogue's release number u (release 0 = initial bias)
+        if (!mbar_wait(&tmem_empty[br.i], br.ph, abort_flag)) { fail(6); break; }
+        tc_fence_after();
+        const uint64_t soff = (uint64_t)((sr.i * Sh::kStageBytes) >> 4);  // descriptor address field: 16-byte units
+        const uint32_t d = tmem_base + br.i * NT;
+        // the buffer holds the bias kAccBias in every element; all four MMAs accumulate onto it
 #pragma unroll
-          for (int k = 0; k < kTileK / 32; ++k)  // K = 32 bytes per instruction: +2 in 16-byte units
-            mma_i8(d, adesc + 2 * k, bdesc + 2 * k, Sh::kIdesc, 1u);
-          mma_commit(&empty[st]);
-          mma_commit(&tmem_full[ab]);
-        }
+        for (int k = 0; k < kTileK / 32; ++k)  // K = 32 bytes per instruction: +2 in 16-byte units
+          mma_i8(d, adesc0 + soff + 2 * k, bdesc0 + soff + 2 * k, Sh::kIdesc, 1u);
+        mma_commit(&empty[sr.i]);
+        mma_commit(&tmem_full[br.i]);
+        sr.next<S_>();
+        br.next<kBufs>();
       }
-      if (!ok && kt > 0) {  // drain the MMAs issued so far
-        const uint32_t last = kt - 1;
-        mbar_wait(&tmem_full[last & 1], (last >> 1) & 1, never_flag);
+      if (g > 0) {  // every MMA issued is complete before tensor memory is freed
+        mma_commit(drain);
+        mbar_wait(drain, 0, never_flag);
       }
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ INT4 expanders
-    const int et = threadIdx.x - 64;  // 0..63
-    uint32_t g = 0, stg_bits = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
-      const Unit x = unit_of(a, u);
-      for (int j = x.j0; j < x.j1; ++j, ++g) {
-        int valid, is4;
-        tile_kinds(a, x.rb, j, valid, is4);
-        if (!is4) continue;
-        const int st = g % S_;
-        if (!mbar_wait(&staged[st], (stg_bits >> st) & 1, abort_flag)) { fail(5); ok = false; break; }
-        stg_bits ^= 1u << st;
-        for (int sub = 0; sub < a.tpb; ++sub) {
-          if (!(is4 >> sub & 1)) continue;
-          const uint8_t* src = stage_g(st) + sub * a.bN * (kTileK / 2);
-          uint8_t* dst = stage_a(st) + sub * a.bN * kTileK;
-          for (int q = et; q < a.bN * 4; q += 64) {  // 16-byte source chunks
-            const int n = q >> 2, c4 = q & 3;
-            const uint4 v = *reinterpret_cast<const uint4*>(src + n * 64 + c4 * 16);
-            const uint2 e0 = expand8_x16(v.x), e1 = expand8_x16(v.y), e2 = expand8_x16(v.z), e3 = expand8_x16(v.w);
-            const int kc0 = 2 * c4, kc1 = 2 * c4 + 1;  // logical 16-byte chunks of the 128-byte row
-            *reinterpret_cast<uint4*>(dst + n * 128 + ((kc0 ^ (n & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-            *reinterpret_cast<uint4*>(dst + n * 128 + ((kc1 ^ (n & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&expanded[st]);
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ tile metadata
+    // Lane l fills the records of tiles g = l, l + 32, ...; the unit and the
+    // tile index `base` where that unit starts follow g forward.
+    uint32_t g = lane;
+    int u = blockIdx.x;
+    uint32_t base = 0;
+    Unit x = unit_of(a, u < a.units ? u : 0);
+    while (u < a.units) {
+      while (u < a.units && g >= base + (uint32_t)(x.j1 - x.j0)) {
+        base += x.j1 - x.j0;
+        u += gridDim.x;
+        if (u < a.units) x = unit_of(a, u);
       }
+      if (u >= a.units) break;
+      const int j = x.j0 + (int)(g - base);
+      const int ms = g % kMetaSlots;
+      if (!mbar_wait(&meta_empty[ms], ((g / kMetaSlots) & 1) ^ 1, abort_flag)) { fail(7); break; }
+      uint32_t kinds = 0, bytes8 = 0, bytes4 = 0, row[2] = {0, 0};
+      for (int sub = 0; sub < a.tpb; ++sub) {
+        const int r = x.rb * a.tpb + sub;
+        if (r < a.R) {
+          const int t = r * a.C + j;
+          const uint32_t is4 = __ldg(a.bitmap + (t >> 3)) >> (t & 7) & 1;
+          kinds |= (1u << (2 + sub)) | (is4 << sub);
+          row[sub] = (uint32_t)__ldg(a.tile_idx + t) * a.bN;
+          if (is4) bytes4 += a.bN * (kTileK / 2);
+          else bytes8 += a.bN * kTileK;
+        }
+      }
+      MetaRec rec;
+      rec.a_row0 = row[0];
+      rec.a_row1 = row[1];
+      rec.sizes = (bytes8 >> 10) | ((bytes4 >> 10) << 8) | (kinds << 28);
+      rec.sc_off = (uint32_t)((x.rb * a.tpb) * a.C + j) * a.bN;
+      meta[ms] = rec;
+      mbar_arrive(&meta_full[ms]);
+      g += kMetaSlots;
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ activation + scale producer
+    if (lane == 0) {
+      const uint32_t g_total = cta_tiles(a);
+      pdl_wait();  // activations come from an earlier kernel
+      TileIter bi(a);
+      RingPos mr{0, 0}, sr{0, 0}, cr{0, 0};
+      bool ok = true;
+      for (uint32_t g = 0; g < g_total; ++g, bi.next(a)) {
+        if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(3); ok = false; break; }
+        mbar_arrive_expect_tx(&full[sr.i], Sh::kB);
+        tma_load_2d(stage_b(sr.i), &tm_x, bi.j * kTileK, bi.x.tb * NT, &full[sr.i]);
+        sr.next<S_>();
+        // the tile's row scales for the epilogue (never waits: the ring is deeper than the pipeline)
+        if (!mbar_wait(&meta_full[mr.i], mr.ph, abort_flag)) { fail(13); ok = false; break; }
+        const uint32_t sizes = meta[mr.i].sizes, sc_off = meta[mr.i].sc_off;
+        mbar_arrive(&meta_empty[mr.i]);
+        mr.next<kMetaSlots>();
+        // No wait for the slot to be free: the slot of tile g was last read for
+        // tile g - kScSlots, and the stage wait above already proves that the
+        // epilogue released tile g - kStages - kBufs >= g - kScSlots (every
+        // epilogue warp reads a tile's scales before releasing its accumulator).
+        const uint32_t kinds = sizes >> 28;
+        sc_info[cr.i] = kinds;
+        uint8_t* dst = sc_ring + cr.i * 256;
+        mbar_arrive_expect_tx(&sc_full[cr.i], (kinds & 8) ? 4u * a.bN : 2u * a.bN);
+        bulk_load(dst, a.scales + sc_off, a.bN * 2, &sc_full[cr.i]);
+        if (kinds & 8) bulk_load(dst + a.bN * 2, a.scales + sc_off + (uint32_t)a.C * a.bN, a.bN * 2, &sc_full[cr.i]);
+        cr.next<kScSlots>();
+      }
+      if (!ok || *abort_flag) abort_grace();
     }
   } else {
     // ------------------------------------------------------------ epilogue
     constexpr int kCols = Sh::kCols;
-    const int ew = warp - 4;
-    const int quad = warp & 3;       // tensor-memory lane quadrant this warp may access
-    const int cg = ew >> 2;          // column group
+    const int ew = warp - kFirstEpiWarp;
+    const int quad = warp & 3;         // tensor-memory lane quadrant this warp may access
+    const int cg = ew >> 2;            // column group
     const int row = 32 * quad + lane;  // row inside the 128-row block
-    const int sub = row / a.bN, nl = row % a.bN;
-    pdl_wait();  // outputs and workspace may still be in use by an earlier kernel
-    // Bias both accumulator buffers: an INT32 sum P accumulated onto 0x4B400000
+    const int sub = row / a.bN;
+    // Bias every accumulator buffer: an INT32 sum P accumulated onto 0x4B400000
     // reads, as an fp32 bit pattern, exactly 12582912 + P for |P| < 2^22, so one
     // fp32 subtraction converts it (no int -> float conversion instruction).
     {
-      const uint32_t lane_base = tmem_base + ((uint32_t)(32 * quad) << 16) + cg * Sh::kCols;
+      const uint32_t lane_base = tmem_base + ((uint32_t)(32 * quad) << 16) + cg * kCols;
 #pragma unroll
-      for (int ab = 0; ab < 2; ++ab)
+      for (int ab = 0; ab < kBufs; ++ab)
 #pragma unroll
-        for (int c16 = 0; c16 < Sh::kCols / 16; ++c16) tmem_st16_const(lane_base + ab * Sh::kBufStride + c16 * 16, kAccBias);
+        for (int c16 = 0; c16 < kCols / 16; ++c16) tmem_st16_const(lane_base + ab * NT + c16 * 16, kAccBias);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&tmem_empty[0]);
-      mbar_arrive(&tmem_empty[1]);
+      __syncwarp();
+      if (lane == 0)
+        for (int ab = 0; ab < kBufs; ++ab) mbar_arrive(&tmem_empty[ab]);
     }
-    uint32_t kt = 0, sync_phase = 0;
-    bool ok = true;
+    // INT4 expansion: tiles ge .. last (this warp's share of each), then
+    // signal the MMA; every warp arrives for every tile, INT4 or not.
+    const int et = threadIdx.x - 32 * kFirstEpiWarp;  // 0 .. 32 kEpiWarps - 1
+    uint32_t g_total = 0;                             // input tiles this CTA processes
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
+      const Unit x = unit_of(a, u);
+      g_total += x.j1 - x.j0;
+    }
+    uint32_t ge = 0;
+    auto expand_upto = [&](uint32_t last) -> bool {
+      for (; ge <= last && ge < g_total; ++ge) {
+        const int st = ge % S_;
+        if (!__all_sync(0xffffffffu, mbar_wait(&staged[st], (ge / S_) & 1, abort_flag))) {
+          fail(8);
+          return false;
+        }
+        const uint32_t info = stage_info[st];
+        const uint32_t is4 = info & (info >> 2) & 3u;
+        for (int sb = 0; sb < a.tpb; ++sb) {
+          if (!(is4 >> sb & 1)) continue;
+          const uint8_t* src = stage_g(st) + sb * a.bN * (kTileK / 2);
+          uint8_t* dst = stage_a(st) + sb * a.bN * kTileK;
+          for (int q = et; q < a.bN * 4; q += 32 * Sh::kEpiWarps) {  // 16-byte source chunks
+            const int r8 = q >> 2, c4 = q & 3;
+            // 32 nibbles -> logical 16-byte chunks 2 c4 and 2 c4 + 1 of the 128-byte row
+            const uint4 v = *reinterpret_cast<const uint4*>(src + r8 * 64 + c4 * 16);
+            uint8_t* drow = dst + r8 * 128;
+            const uint2 e0 = expand8_x16(v.x), e1 = expand8_x16(v.y);
+            *reinterpret_cast<uint4*>(drow + (((2 * c4) ^ (r8 & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+            const uint2 e2 = expand8_x16(v.z), e3 = expand8_x16(v.w);
+            *reinterpret_cast<uint4*>(drow + (((2 * c4 + 1) ^ (r8 & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+          }
+        }
+        if (is4) fence_proxy_async_smem();  // generic-proxy writes -> visible to the MMA's async proxy
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&expanded[st]);
+      }
+      return true;
+    };
+    bool ok = expand_upto(kExpandAhead - 1);  // weights only: may overlap the previous kernel
+    pdl_wait();  // outputs, token scales and workspace may still be in use by an earlier kernel
+    const float2 nbias = make_float2(-kAccBiasF, -kAccBiasF);
+    uint32_t g = 0, sync_phase = 0;
     for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
       const Unit x = unit_of(a, u);
-      const int r = x.rb * a.tpb + sub;
-      const bool rvalid = r < a.R;
-      const int n = r * a.bN + nl;
+      const int n = x.rb * 128 + row;  // output feature of this thread
+      const bool rvalid = n < a.N;
       const int mcol0 = x.tb * NT + cg * kCols;  // first token of this thread's columns
-      float acc[kCols];
-#pragma unroll
-      for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
-      // tile scale and kind of the next input tile are loaded one tile ahead
-      auto load_scale = [&](int j, uint32_t& swb, uint32_t& lab) {
-        if (rvalid) {
-          const int tt = r * a.C + j;
-          swb = __ldg(a.scales + (size_t)tt * a.bN + nl);
-          lab = __ldg(a.bitmap + (tt >> 3)) >> (tt & 7);
+      // bias of this row and the token scales of the warp's columns, copied
+      // into shared memory now and read at the end of the unit
+      if constexpr (MODE != 2) {
+        const bool has_b = rvalid && a.bias != nullptr;
+        cp_async4(pre_bias + et, has_b ? a.bias + n : a.sx, has_b ? 4u : 0u);
+        for (int c = lane; c < kCols; c += 32) {
+          const bool has_s = mcol0 + c < a.M;
+          cp_async4(pre_sx + ew * kCols + c, has_s ? a.sx + mcol0 + c : a.sx, has_s ? 4u : 0u);
         }
-      };
-      uint32_t swb_next = 0, lab_next = 0;
-      load_scale(x.j0, swb_next, lab_next);
-      for (int j = x.j0; j < x.j1; ++j, ++kt) {
-        const int ab = kt & 1;
-        const uint32_t swb = swb_next, lab = lab_next;
-        if (j + 1 < x.j1) load_scale(j + 1, swb_next, lab_next);
-        // INT4 tiles were multiplied by 16 during expansion
-        const bool t4 = rvalid && (lab & 1);
-        const float sw = rvalid ? __half2float(__ushort_as_half((unsigned short)swb)) * (t4 ? 0.0625f : 1.0f) : 0.f;
-        // warp-uniform outcome: the tensor-memory loads below are warp-collective
-        if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[ab], (kt >> 1) & 1, abort_flag))) {
-          fail(6);
+        cp_async_commit();
+      }
+      float2 acc[kCols / 2];
+#pragma unroll
+      for (int i = 0; i < kCols / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+      for (int j = x.j0; j < x.j1; ++j, ++g) {
+        const int sl = g % kScSlots, ab = g % kBufs;
+        // the tile's row scales and its INT32 products (warp-uniform outcome: the
+        // tensor-memory loads below are warp-collective)
+        if (!__all_sync(0xffffffffu, mbar_wait(&sc_full[sl], (g / kScSlots) & 1, abort_flag) &&
+                                         mbar_wait(&tmem_full[ab], (g / kBufs) & 1, abort_flag))) {
+          fail(9);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + ab * Sh::kBufStride + cg * kCols;
+        const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + ab * NT + cg * kCols;
+        uint32_t v[Sh::kLdCols];
 #pragma unroll
-        for (int c16 = 0; c16 < kCols / 16; ++c16) {
-          uint32_t v[16];
-          tmem_ld16(taddr + c16 * 16, v);
+        for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
+          tmem_ld16(taddr + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
+        // while the first loads are in flight: the weight scale, and the INT4
+        // expansion of a later tile
+        const bool t4 = (sc_info[sl] >> sub) & 1;
+        const uint16_t swb = reinterpret_cast<const uint16_t*>(sc_ring + sl * 256)[row];
+        // INT4 tiles were multiplied by 16 during expansion
+        const float sw = rvalid ? __half2float(__ushort_as_half(swb)) * (t4 ? 0.0625f : 1.0f) : 0.f;
+        const float2 sw2 = make_float2(sw, sw);
+        const bool eok = expand_upto(g + kExpandAhead);
+#pragma unroll
+        for (int c0 = 0; c0 < kCols; c0 += Sh::kLdCols) {
+          if (c0 > 0) {
+#pragma unroll
+            for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
+              tmem_ld16(taddr + c0 + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
+          }
           tmem_wait_ld();
-          tmem_st16_const(taddr + c16 * 16, kAccBias);  // re-bias for the buffer's next use
+#pragma unroll
+          for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16) tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
+#pragma unroll
+          for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
+            tmem_st16_const(taddr + c0 + c16 * 16, kAccBias);  // re-bias for the buffer's next use
           if constexpr (MODE == 2) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int m = mcol0 + c16 * 16 + i;
+            for (int i = 0; i < Sh::kLdCols; ++i) {
+              const int m = mcol0 + c0 + i;
               if (rvalid && m < a.M) {
                 const int p16 = (int)(v[i] - kAccBias);
                 a.P[((size_t)m * a.N + n) * a.C + j] = t4 ? (p16 >> 4) : p16;
@@ -375,24 +588,55 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
             }
           } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              acc[c16 * 16 + i] = fmaf(__uint_as_float(v[i]) - kAccBiasF, sw, acc[c16 * 16 + i]);
+            for (int i = 0; i < Sh::kLdCols / 2; ++i) {
+              const float2 p = __fadd2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), nbias);
+              acc[c0 / 2 + i] = __ffma2_rn(p, sw2, acc[c0 / 2 + i]);
+            }
           }
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&tmem_empty[ab]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tmem_empty[ab]);
+        if (!eok) {
+          ok = false;
+          break;
+        }
       }
       if (!ok || MODE == 2) continue;
+      cp_async_wait_all();
+      __syncwarp();  // the token scales were copied by all lanes of the warp
+      const float bias_n = pre_bias[et];
       if constexpr (MODE == 0) {
-        if (rvalid) {
-          const float b = a.bias ? __ldg(a.bias + n) : 0.f;
+        const float4* sxv = reinterpret_cast<const float4*>(pre_sx + ew * kCols);
+        const int mlim = a.M - mcol0;  // columns of this thread that exist
+        if (rvalid && a.ydtype == AQ_F32) {
+          float* yp = reinterpret_cast<float*>(a.y) + (size_t)mcol0 * a.ldy + n;
 #pragma unroll
-          for (int i = 0; i < kCols; ++i) {
-            const int m = mcol0 + i;
-            if (m < a.M) store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), acc[i], b));
+          for (int i4 = 0; i4 < kCols / 4; ++i4) {
+            const float4 s4 = sxv[i4];
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = 4 * i4 + k;
+              if (i < mlim) yp[(size_t)i * a.ldy] = fmaf(sv[k], i & 1 ? acc[i / 2].y : acc[i / 2].x, bias_n);
+            }
+          }
+        } else if (rvalid) {
+          __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(a.y) + (size_t)mcol0 * a.ldy + n;
+#pragma unroll
+          for (int i4 = 0; i4 < kCols / 4; ++i4) {
+            const float4 s4 = sxv[i4];
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = 4 * i4 + k;
+              if (i < mlim)
+                yp[(size_t)i * a.ldy] = __float2bfloat16_rn(fmaf(sv[k], i & 1 ? acc[i / 2].y : acc[i / 2].x, bias_n));
+            }
           }
         }
+        __syncwarp();  // the scale slots are rewritten at the next unit's start
         continue;
       }
       // split-K: publish the partial sum, the last CTA of this unit group reduces
@@ -400,32 +644,33 @@ __global__ void __launch_bounds__(TcShape<NT>::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kCols; ++i) {
           const int m = mcol0 + i;
-          if (m < a.M) __stcg(a.partial + ((size_t)x.s * a.M + m) * a.N + n, acc[i]);
+          const float s = i & 1 ? acc[i / 2].y : acc[i / 2].x;
+          if (m < a.M) __stcg(a.partial + ((size_t)x.s * a.M + m) * a.N + n, s);
         }
       }
       __threadfence();
       mbar_arrive(epi_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag))) { fail(7); ok = false; continue; }
+      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag))) { fail(11); ok = false; continue; }
       sync_phase ^= 1;
       if (ew == 0 && lane == 0) *last_flag = (atomicAdd(a.counters + x.rb * a.ntb + x.tb, 1) == a.S - 1);
       mbar_arrive(epi_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag))) { fail(8); ok = false; continue; }
+      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag))) { fail(12); ok = false; continue; }
       sync_phase ^= 1;
       if (*last_flag) {
         __threadfence();
         if (rvalid) {
-          const float b = a.bias ? __ldg(a.bias + n) : 0.f;
           for (int i = 0; i < kCols; ++i) {
             const int m = mcol0 + i;
             if (m >= a.M) break;
             float sum = 0.f;
             for (int ss = 0; ss < a.S; ++ss) sum += __ldcg(a.partial + ((size_t)ss * a.M + m) * a.N + n);
-            store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sum, b));
+            store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sum, bias_n));
           }
         }
         if (ew == 0 && lane == 0) a.counters[x.rb * a.ntb + x.tb] = 0;
       }
     }
+    cp_async_wait_all();  // no copy into shared memory outlives the CTA (abort path)
   }
 
   tc_fence_before();
@@ -505,11 +750,8 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
   char* wsb = static_cast<char*>(ws);
   a.counters = reinterpret_cast<int*>(wsb + kWsHeader);
 
-  int nt;
-  if (phase == AQ_PHASE_DECODE || M <= 64) nt = (M + 15) / 16 * 16;
-  else if (M <= 128) nt = 128;
-  else nt = 256;
-  if (nt > 64 && nt < 128) nt = 128;
+  // token-block width: up to 64 tokens in one block of 16-multiples, 128 beyond
+  const int nt = M <= 64 ? (M + 15) / 16 * 16 : 128;
   a.ntb = (M + nt - 1) / nt;
   if (phase == AQ_PHASE_DECODE && P == nullptr) {
     const DecodePlan p = plan_decode(M, w);
@@ -533,8 +775,6 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
     AQ_TC_CASE(48)
     AQ_TC_CASE(64)
     AQ_TC_CASE(128)
-    case 256 * 4 + 0: return launch_nt<256, 0>(w, xq, a, grid, st);
-    case 256 * 4 + 2: return launch_nt<256, 2>(w, xq, a, grid, st);
 #undef AQ_TC_CASE
     default: return cudaErrorInvalidValue;
   }
