@@ -120,21 +120,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Like mbar_try_wait, but a thread whose phase is not complete sleeps in
+// hardware until it completes or kWaitSuspendNs pass, instead of spinning
+// (spinning waiters take issue slots from the warps doing the work).
+constexpr uint32_t kWaitSuspendNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false when
-// `abort` became nonzero or the time limit passed; never spins unbounded.
-// Reading %globaltimer costs hundreds of nanoseconds, so the clock (and the
-// abort flag) are checked only every 256 unsuccessful polls.
+// `abort` became nonzero or the time limit passed; never waits unbounded.
+// Between checks of the abort flag and the clock the thread sleeps (see
+// mbar_try_wait_sleep), so the checks cost little.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = 0;
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 255u) == 0) {
-      if (*abort) return false;
-      const unsigned long long now = globaltimer_ns();
-      if (t0 == 0) t0 = now;
-      else if (now - t0 > kWaitTimeoutNs) return false;
-    }
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
   }
 }
 

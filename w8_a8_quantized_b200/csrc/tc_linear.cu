@@ -9,7 +9,8 @@
 // Roles in one CTA (persistent over work units; every role walks the same
 // sequence of input tiles g = 0, 1, 2, ... of the CTA's units):
 //   warp 0      weight producer: INT8 tiles -> swizzled A stage (TMA), INT4
-//               tiles -> staging buffer (TMA).  It does not wait for the
+//               tiles -> staging buffer (TMA), the tile's fp16 row scales ->
+//               the stage's scale area (bulk copy).  It does not wait for the
 //               previous kernel, so the first stages load while it finishes.
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma
 //               (kind::i8, M = 128 weight rows, N = NT tokens, K = 32) four
@@ -21,8 +22,7 @@
 //               ring, so the producers spend a handful of instructions per tile.
 //   warp 3      activation producer: the NT x 128 INT8 activation tile -> B
 //               stage (TMA), after the previous kernel (which writes the
-//               activations) is done; and the tile's fp16 row scales -> scale
-//               ring (bulk copy) for the epilogue.
+//               activations) is done.
 //   warps 4..   epilogue; warp w may read tensor-memory lanes 32 (w % 4) ..
 //               32 (w % 4) + 31.  After every input tile it reads the INT32
 //               tile product from tensor memory, multiplies by the row's fp16
@@ -32,9 +32,10 @@
 //               The same warps expand the INT4 staging tiles into the
 //               128-byte-swizzled INT8 A layout kExpandAhead tiles ahead of
 //               the tile they rescale (fence.proxy.async before signalling the
-//               MMA): expansion runs on the integer and load/store pipes beside
-//               the FP32 rescale, and no separate expander warps take
-//               registers from the epilogue.
+//               MMA), and at that point copy their row's weight scale of the
+//               tile into a private shared-memory ring, so the rescale itself
+//               waits on nothing but the accumulator.  Tiles are rescaled in
+//               pairs: one accumulator wait and one release per two tiles.
 // A single thread on a busy SM retires roughly one dependent instruction every
 // 10-20 cycles, so the per-tile work of each issuing thread is kept to a few
 // dozen instructions and spread over three threads.
@@ -64,13 +65,13 @@ namespace aq {
 namespace {
 
 constexpr int kBufs = 4;        // accumulator buffers in tensor memory
-constexpr int kScSlots = 16;    // scale ring slots (>= stages + kBufs: slots are reused without a barrier)
+constexpr int kSwRing = 8;      // per-thread ring of expanded-ahead weight scales (> kExpandAhead + 1)
 constexpr int kMetaSlots = 32;  // metadata ring slots (one per lane of the metadata warp)
 constexpr int kFirstEpiWarp = 4;
 // Tiles the epilogue expands ahead of the one it rescales.  At least kBufs,
 // so the MMA (at most kBufs tiles ahead of the epilogue) never waits for an
-// expansion; below stages + kBufs, so the staging copy it waits for never
-// depends on the epilogue's own later progress.
+// expansion; below stages + kBufs (counting the second tile of a pair), so the
+// staging copy it waits for never depends on the epilogue's own later progress.
 constexpr int kExpandAhead = kBufs;
 
 template <int NT>
@@ -95,16 +96,20 @@ struct TcShape {
   static constexpr int kMaxRegs = kMaxRegsRaw > 255 ? 255 : kMaxRegsRaw;
   static constexpr int kTmemCols = kBufs * NT <= 32 ? 32 : kBufs * NT <= 64 ? 64 : kBufs * NT <= 128 ? 128
                                    : kBufs * NT <= 256 ? 256 : 512;
-  static constexpr int kScBytes = kScSlots * 256;  // 128 rows x fp16 per slot
+  static constexpr int kScBytes = kStages * 256;  // per stage: the tile's 128 row scales (fp16)
+  static constexpr int kSwBytes = kSwRing * 32 * kEpiWarps * 4;  // [kSwRing][epilogue thread] fp32
   static constexpr int kCtrlBytes = 2048;
   static constexpr int kPreBytes = (32 + kCols) * kEpiWarps * 4;  // per-unit bias and token scales of the epilogue
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kScBytes + kCtrlBytes + kPreBytes;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kScBytes + kCtrlBytes + kPreBytes + kSwBytes;
   static constexpr uint32_t kIdesc = idesc_i8(128, NT);
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= 128, "MMA N");
   static_assert(kBufs * NT <= 512, "tensor memory");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
-  static_assert(kStages >= 3 && kScSlots >= kStages + kBufs, "ring depths");
-  static_assert(kExpandAhead >= kBufs && kExpandAhead < kStages + kBufs, "expansion distance");
+  static_assert(kStages >= 3, "ring depth");
+  // pairs of tiles: the epilogue expands up to tile g + 1 + kExpandAhead while
+  // it still holds tile g
+  static_assert(kExpandAhead >= kBufs && kExpandAhead + 1 < kStages + kBufs, "expansion distance");
+  static_assert(kSwRing > kExpandAhead + 1, "scale ring depth");
   static_assert(kThreads <= 1024, "block size");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -259,29 +264,28 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
   auto stage_a = [&](int st) { return smem + st * Sh::kStageBytes; };
   auto stage_b = [&](int st) { return smem + st * Sh::kStageBytes + Sh::kA; };
   auto stage_g = [&](int st) { return smem + st * Sh::kStageBytes + Sh::kA + Sh::kB; };
-  uint8_t* sc_ring = smem + S_ * Sh::kStageBytes;  // [kScSlots][128] fp16
-  uint8_t* ctrl = sc_ring + Sh::kScBytes;
+  uint8_t* stage_sc = smem + S_ * Sh::kStageBytes;  // [stage][128] fp16 row scales
+  uint8_t* ctrl = stage_sc + Sh::kScBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);  // weights (INT8) + activations landed; one arrival per producer
   uint64_t* staged = full + S_;                        // INT4 staging landed (0 bytes when none)
   uint64_t* expanded = staged + S_;                    // epilogue warps done expanding the stage (one arrival each)
   uint64_t* empty = expanded + S_;                     // MMAs reading the stage done
   uint64_t* tmem_full = empty + S_;
   uint64_t* tmem_empty = tmem_full + kBufs;
-  uint64_t* sc_full = tmem_empty + kBufs;
-  uint64_t* meta_full = sc_full + kScSlots;
+  uint64_t* meta_full = tmem_empty + kBufs;
   uint64_t* meta_empty = meta_full + kMetaSlots;
   uint64_t* epi_sync = meta_empty + kMetaSlots;  // epilogue-only rendezvous (bounded, unlike bar.sync)
   uint64_t* drain = epi_sync + 1;                // MMA completion on the way out
   MetaRec* meta = reinterpret_cast<MetaRec*>(drain + 1);
   volatile uint32_t* stage_info = reinterpret_cast<volatile uint32_t*>(meta + kMetaSlots);
-  volatile uint32_t* sc_info = stage_info + S_;
-  uint32_t* tmem_slot = const_cast<uint32_t*>(sc_info + kScSlots);
+  uint32_t* tmem_slot = const_cast<uint32_t*>(stage_info + S_);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
   volatile int* never_flag = reinterpret_cast<volatile int*>(tmem_slot + 3);  // stays 0: drain waits
   float* pre_bias = reinterpret_cast<float*>(ctrl + Sh::kCtrlBytes);  // [32 kEpiWarps] bias of each epilogue row
   float* pre_sx = pre_bias + 32 * Sh::kEpiWarps;                       // [kEpiWarps][kCols] token scales
-  static_assert((4 * 8 + 2 * kBufs + 2 * kScSlots + 2 * kMetaSlots + 2) * 8 + kMetaSlots * 16 + (8 + kScSlots + 4) * 4 <=
+  float* pre_sw = pre_sx + Sh::kEpiWarps * Sh::kCols;                    // [kSwRing][32 kEpiWarps] weight scales
+  static_assert((4 * 8 + 2 * kBufs + 2 * kMetaSlots + 2) * 8 + kMetaSlots * 16 + (8 + 4) * 4 <=
                     Sh::kCtrlBytes,
                 "control area");
 
@@ -297,12 +301,9 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       mbar_init(&tmem_full[b], 1);
       mbar_init(&tmem_empty[b], Sh::kEpiWarps);
     }
-    for (int s = 0; s < kScSlots; ++s) {
-      mbar_init(&sc_full[s], 1);
-    }
     for (int s = 0; s < kMetaSlots; ++s) {
       mbar_init(&meta_full[s], 1);
-      mbar_init(&meta_empty[s], 2);  // both producers read every record
+      mbar_init(&meta_empty[s], 1);
     }
     mbar_init(epi_sync, 32 * Sh::kEpiWarps);
     mbar_init(drain, 1);
@@ -341,9 +342,13 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         mr.next<kMetaSlots>();
         if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(2); ok = false; break; }
         const uint32_t kinds = rec.sizes >> 28;
+        const uint32_t sc_bytes = (kinds & 8) ? 4u * a.bN : 2u * a.bN;  // fp16 row scales of the tile's sub-tiles
         stage_info[sr.i] = kinds;  // read by the expanding epilogue warps after `staged`
         mbar_arrive_expect_tx(&full[sr.i], (rec.sizes & 0xFFu) << 10);
-        mbar_arrive_expect_tx(&staged[sr.i], ((rec.sizes >> 8) & 0xFFu) << 10);
+        mbar_arrive_expect_tx(&staged[sr.i], (((rec.sizes >> 8) & 0xFFu) << 10) + sc_bytes);
+        uint8_t* scd = stage_sc + sr.i * 256;
+        bulk_load(scd, a.scales + rec.sc_off, a.bN * 2, &staged[sr.i]);
+        if (kinds & 8) bulk_load(scd + a.bN * 2, a.scales + rec.sc_off + (uint32_t)a.C * a.bN, a.bN * 2, &staged[sr.i]);
         if (kinds & 1) tma_load_2d(stage_g(sr.i), &tm_w4, 0, rec.a_row0, &staged[sr.i]);
         else tma_load_2d(stage_a(sr.i), &tm_w8, 0, rec.a_row0, &full[sr.i]);
         if (kinds & 8) {
@@ -424,34 +429,18 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       g += kMetaSlots;
     }
   } else if (warp == 3) {
-    // ------------------------------------------------------------ activation + scale producer
+    // ------------------------------------------------------------ activation producer
     if (lane == 0) {
       const uint32_t g_total = cta_tiles(a);
       pdl_wait();  // activations come from an earlier kernel
       TileIter bi(a);
-      RingPos mr{0, 0}, sr{0, 0}, cr{0, 0};
+      RingPos sr{0, 0};
       bool ok = true;
       for (uint32_t g = 0; g < g_total; ++g, bi.next(a)) {
         if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(3); ok = false; break; }
         mbar_arrive_expect_tx(&full[sr.i], Sh::kB);
         tma_load_2d(stage_b(sr.i), &tm_x, bi.j * kTileK, bi.x.tb * NT, &full[sr.i]);
         sr.next<S_>();
-        // the tile's row scales for the epilogue (never waits: the ring is deeper than the pipeline)
-        if (!mbar_wait(&meta_full[mr.i], mr.ph, abort_flag)) { fail(13); ok = false; break; }
-        const uint32_t sizes = meta[mr.i].sizes, sc_off = meta[mr.i].sc_off;
-        mbar_arrive(&meta_empty[mr.i]);
-        mr.next<kMetaSlots>();
-        // No wait for the slot to be free: the slot of tile g was last read for
-        // tile g - kScSlots, and the stage wait above already proves that the
-        // epilogue released tile g - kStages - kBufs >= g - kScSlots (every
-        // epilogue warp reads a tile's scales before releasing its accumulator).
-        const uint32_t kinds = sizes >> 28;
-        sc_info[cr.i] = kinds;
-        uint8_t* dst = sc_ring + cr.i * 256;
-        mbar_arrive_expect_tx(&sc_full[cr.i], (kinds & 8) ? 4u * a.bN : 2u * a.bN);
-        bulk_load(dst, a.scales + sc_off, a.bN * 2, &sc_full[cr.i]);
-        if (kinds & 8) bulk_load(dst + a.bN * 2, a.scales + sc_off + (uint32_t)a.C * a.bN, a.bN * 2, &sc_full[cr.i]);
-        cr.next<kScSlots>();
       }
       if (!ok || *abort_flag) abort_grace();
     }
@@ -479,7 +468,9 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         for (int ab = 0; ab < kBufs; ++ab) mbar_arrive(&tmem_empty[ab]);
     }
     // INT4 expansion: tiles ge .. last (this warp's share of each), then
-    // signal the MMA; every warp arrives for every tile, INT4 or not.
+    // signal the MMA; every warp arrives for every tile, INT4 or not.  Each
+    // thread also stashes its row's weight scale of the tile (0 for a row past
+    // the layer's end; / 16 for INT4, whose codes were expanded as 16 q).
     const int et = threadIdx.x - 32 * kFirstEpiWarp;  // 0 .. 32 kEpiWarps - 1
     uint32_t g_total = 0;                             // input tiles this CTA processes
     for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
@@ -496,6 +487,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         }
         const uint32_t info = stage_info[st];
         const uint32_t is4 = info & (info >> 2) & 3u;
+        {
+          const float swv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(stage_sc + st * 256)[row]));
+          pre_sw[(ge % kSwRing) * 32 * Sh::kEpiWarps + et] =
+              (info >> (2 + sub) & 1) ? swv * ((is4 >> sub & 1) ? 0.0625f : 1.0f) : 0.f;
+        }
         for (int sb = 0; sb < a.tpb; ++sb) {
           if (!(is4 >> sb & 1)) continue;
           const uint8_t* src = stage_g(st) + sb * a.bN * (kTileK / 2);
@@ -540,64 +536,72 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       float2 acc[kCols / 2];
 #pragma unroll
       for (int i = 0; i < kCols / 2; ++i) acc[i] = make_float2(0.f, 0.f);
-      for (int j = x.j0; j < x.j1; ++j, ++g) {
-        const int sl = g % kScSlots, ab = g % kBufs;
-        // the tile's row scales and its INT32 products (warp-uniform outcome: the
-        // tensor-memory loads below are warp-collective)
-        if (!__all_sync(0xffffffffu, mbar_wait(&sc_full[sl], (g / kScSlots) & 1, abort_flag) &&
-                                         mbar_wait(&tmem_full[ab], (g / kBufs) & 1, abort_flag))) {
+      for (int j = x.j0; j < x.j1;) {
+        // a pair of tiles (the last one of an odd unit alone): the commit of the
+        // second tile's MMAs follows the first's, so one wait covers both
+        const int nt = j + 1 < x.j1 ? 2 : 1;
+        const uint32_t gl = g + nt - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[gl % kBufs], (gl / kBufs) & 1, abort_flag))) {
           fail(9);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + ab * NT + cg * kCols;
-        uint32_t v[Sh::kLdCols];
-#pragma unroll
-        for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
-          tmem_ld16(taddr + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
-        // while the first loads are in flight: the weight scale, and the INT4
-        // expansion of a later tile
-        const bool t4 = (sc_info[sl] >> sub) & 1;
-        const uint16_t swb = reinterpret_cast<const uint16_t*>(sc_ring + sl * 256)[row];
-        // INT4 tiles were multiplied by 16 during expansion
-        const float sw = rvalid ? __half2float(__ushort_as_half(swb)) * (t4 ? 0.0625f : 1.0f) : 0.f;
-        const float2 sw2 = make_float2(sw, sw);
-        const bool eok = expand_upto(g + kExpandAhead);
-#pragma unroll
-        for (int c0 = 0; c0 < kCols; c0 += Sh::kLdCols) {
-          if (c0 > 0) {
-#pragma unroll
-            for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
-              tmem_ld16(taddr + c0 + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
-          }
-          tmem_wait_ld();
-#pragma unroll
-          for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16) tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
+        bool eok = true;
+        for (int k = 0; k < nt; ++k) {
+          const uint32_t gk = g + k;
+          const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (gk % kBufs) * NT + cg * kCols;
+          uint32_t v[Sh::kLdCols];
 #pragma unroll
           for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
-            tmem_st16_const(taddr + c0 + c16 * 16, kAccBias);  // re-bias for the buffer's next use
-          if constexpr (MODE == 2) {
+            tmem_ld16(taddr + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
+          // while the first loads are in flight: the INT4 expansion of later tiles
+          if (k == 0) eok = expand_upto(gl + kExpandAhead);
+          const float sw = pre_sw[(gk % kSwRing) * 32 * Sh::kEpiWarps + et];
+          const float2 sw2 = make_float2(sw, sw);
 #pragma unroll
-            for (int i = 0; i < Sh::kLdCols; ++i) {
-              const int m = mcol0 + c0 + i;
-              if (rvalid && m < a.M) {
-                const int p16 = (int)(v[i] - kAccBias);
-                a.P[((size_t)m * a.N + n) * a.C + j] = t4 ? (p16 >> 4) : p16;
-              }
+          for (int c0 = 0; c0 < kCols; c0 += Sh::kLdCols) {
+            if (c0 > 0) {
+#pragma unroll
+              for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
+                tmem_ld16(taddr + c0 + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
             }
-          } else {
+            tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < Sh::kLdCols / 2; ++i) {
-              const float2 p = __fadd2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), nbias);
-              acc[c0 / 2 + i] = __ffma2_rn(p, sw2, acc[c0 / 2 + i]);
+            for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16) tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
+#pragma unroll
+            for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
+              tmem_st16_const(taddr + c0 + c16 * 16, kAccBias);  // re-bias for the buffer's next use
+            if constexpr (MODE == 2) {
+              // INT4 label read back from the bitmap (debug path only)
+              const int tt = (n / a.bN) * a.C + j + k;
+              const bool t4 = rvalid && ((__ldg(a.bitmap + (tt >> 3)) >> (tt & 7)) & 1);
+#pragma unroll
+              for (int i = 0; i < Sh::kLdCols; ++i) {
+                const int m = mcol0 + c0 + i;
+                if (rvalid && m < a.M) {
+                  const int p16 = (int)(v[i] - kAccBias);
+                  a.P[((size_t)m * a.N + n) * a.C + j + k] = t4 ? (p16 >> 4) : p16;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < Sh::kLdCols / 2; ++i) {
+                const float2 p = __fadd2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), nbias);
+                acc[c0 / 2 + i] = __ffma2_rn(p, sw2, acc[c0 / 2 + i]);
+              }
             }
           }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tmem_empty[ab]);
+        if (lane == 0) {
+          mbar_arrive(&tmem_empty[g % kBufs]);
+          if (nt == 2) mbar_arrive(&tmem_empty[gl % kBufs]);
+        }
+        g += nt;
+        j += nt;
         if (!eok) {
           ok = false;
           break;
