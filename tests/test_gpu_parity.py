@@ -205,6 +205,18 @@ def _group_case(shapes, M, seed, phase, bN=128, frac8=0.25):
     return ps, ws, x
 
 
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_decode_wide_layer_matches_oracle(M):
+    """A layer wider than one 32-row CUDA-core block per SM (so blocks queue
+    behind each other); bf16 output, with bias."""
+    N, K = 4864, 1024
+    p, x, w, xq, sx = packed_case(N, K, 128, 0.25, 1200 + M, M, outlier=0.01)
+    bias = np.linspace(-1, 1, N).astype(np.float32)
+    y = aq.aq_linear_decode(w, xq, sx, bias=torch.from_numpy(bias).cuda(), out_dtype=torch.bfloat16)
+    assert_output_close(y, oracle_linear(p, x, bias=bias))
+    aq.check_all_workspaces()
+
+
 @pytest.mark.parametrize("M", [1, 2, 5, 8, 9, 24, 64])
 def test_group_decode_matches_separate_calls_and_oracle(M):
     shapes = [(768, 1024), (256, 1024), (256, 1024)]

@@ -176,7 +176,6 @@ struct TileIter {
     ++j;
     skip(a);
   }
-  __device__ __forceinline__ bool valid(const TcArgs& a) const { return u < a.units; }
 };
 
 // Per-tile record of the metadata ring: everything the producers need to
