@@ -63,6 +63,12 @@ struct RowsArgs {
 
 __device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) { return __dp4a((int)a, (int)b, c); }
 
+// Start moving `bytes` (a multiple of 16, 16-byte aligned) from HBM into L2;
+// no shared memory, no completion to wait for.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes) : "memory");
+}
+
 // Exact int -> float for |v| < 2^22 with an integer add and a float subtract.
 __device__ __forceinline__ float small_int_to_float(int v) {
   return __int_as_float(v + 0x4B400000) - 12582912.0f;
@@ -154,6 +160,13 @@ __global__ void __launch_bounds__(kMaxThreads) decode_rows_kernel(const __grid_c
   }
   __syncthreads();
   pdl_launch_dependents();
+  // the CTA's whole weight slice starts streaming into L2 now, so the DRAM
+  // transfer overlaps the activation preparation below and the register ring
+  // reads from L2
+  for (int j = t; j < C; j += nthr) {
+    const bool is4 = (tile_is4[j >> 5] >> (j & 31)) & 1;
+    prefetch_l2_bulk(tile_ptr[j], kRows * (is4 ? kTileK / 2 : kTileK));
+  }
 
   // ---- this thread's piece of its i-th tile column (j = kg + KG i)
   auto load = [&](int i, Piece& pc) {
