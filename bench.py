@@ -58,10 +58,10 @@ WORKLOADS = {
 # from the ncu captures summarised in profiles/, valid only while the kernel source is unchanged
 # (sha256 prefix of the source file and the shared header).
 MEASURED_TRAFFIC = {
-    # profiles/decode_rows_llama3b_1token.md: one layer's four launches read 64,728,320 B and wrote
-    # 5,120 B -> 16,183,360 B per launch (algorithmic: 16,128,638 B per launch)
+    # profiles/decode_rows_llama3b_1token.md: one layer's four launches read 64,739,840 B and wrote
+    # 43,008 B -> 16,195,712 B per launch (algorithmic: 16,128,638 B per launch)
     "decode": {"src": ("w8_a8_quantized_b200/csrc/decode_rows.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
-               "sha": "75c2b2e21933c4bb", "bytes_per_launch": 16183360},
+               "sha": "bd490b45652ac896", "bytes_per_launch": 16195712},
     "prefill": {"src": ("w8_a8_quantized_b200/csrc/tc_linear.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
                 "sha": None, "bytes_per_launch": None},
 }
@@ -95,6 +95,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="measure only this token count")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="build only the first N layers (small cases for profiling; the line records the count)")
     return ap.parse_args()
 
 
@@ -166,14 +168,14 @@ class ClockSampler:
 class Model:
     """Packed random weights and synthetic activations of one workload on one GPU."""
 
-    def __init__(self, wl: dict, M: int, device, rank: int):
+    def __init__(self, wl: dict, M: int, device, rank: int, layers=None):
         import torch
         from w8_a8_quantized_b200 import aq, synth
         self.torch, self.aq = torch, aq
         self.wl, self.M, self.dev = wl, M, device
         model = wl["model"]
         cfg = CFG_ID[model]
-        self.layers = synth.MODELS[model]["layers"]
+        self.layers = synth.MODELS[model]["layers"] if layers is None else min(layers, synth.MODELS[model]["layers"])
         self.projs = synth.projections(model)
         self.weights = []
         self.weight_bytes = 0
@@ -397,7 +399,7 @@ def main():
 
     Ms = [wl["M"], *wl["extra_M"]] if args.tokens is None else [args.tokens]
     t_setup = time.time()
-    model = Model(wl, Ms[0], dev, rank)
+    model = Model(wl, Ms[0], dev, rank, args.layers)
     setup_s = time.time() - t_setup
 
     results = {}
@@ -464,7 +466,9 @@ def main():
         "config": {"workload": args.workload, "model_shape": wl["model"], "phase": wl["phase"], "tokens": Ms[0],
                    "tile": [wl["bN"], 128], "int8_tile_fraction": wl["frac8"], "layers": model.layers,
                    "projections_per_layer": 7, "packed_weight_bytes": wbytes, "parallelism": f"replicas x{world}",
-                   "l2": "not flushed: weights streamed per step exceed the 126 MB L2", "graph": "one CUDA graph per step"},
+                   "l2": ("not flushed: weights streamed per step exceed the 126 MB L2" if wbytes > 126e6 else
+                          "not flushed: weights of a reduced --layers case may stay in L2 (profiling only)"),
+                   "graph": "one CUDA graph per step"},
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": r0["h2d"], "d2h_bytes_per_step": r0["d2h"]},
         "gpu_launches": r0["launches"] * args.steps,
         "roofline": roof,
@@ -484,7 +488,7 @@ def main():
 
     if decode and not args.no_prefill and args.workload == "decode-llama-3.2-3b":
         pwl = WORKLOADS["prefill-qwen3-4b"]
-        pm = Model(pwl, pwl["M"], dev, rank)
+        pm = Model(pwl, pwl["M"], dev, rank, args.layers)
         g, launches = pm.graph()
         ms = time_graph(torch, g, max(3, args.steps // 2), max(3, args.warmup), dist_on, dev)
         pm.quantize_inputs()
