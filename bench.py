@@ -87,7 +87,7 @@ INPUT_OF = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out", "ga
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)  # ~0.25 s timed at 1 token: several clock samples
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="aq", choices=["aq", "reference"])
     ap.add_argument("--workload", default="decode-llama-3.2-3b", choices=sorted(WORKLOADS))
