@@ -21,6 +21,12 @@ int validate_packed(const aq_packed* w) {
 
 static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
+// Fusing the activation preparation into every CTA of the CUDA-core decode
+// kernel pays off for 1-2 tokens; from 4 tokens on, one preparation kernel plus
+// a single grouped launch over pre-quantized codes is faster (the per-CTA
+// preparation grows with M).  The fused codes live in shared memory.
+bool rows_fusable(int M, int K) { return M <= 2 && 2 * (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
+
 // Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, one CTA per 16
 // output rows, no split); more tokens on the tensor cores with splits over
 // tile columns to fill the GPU.
@@ -220,7 +226,8 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
     e = launch_decode_rows(d, G, K, x, ldx, nullptr, nullptr, M, ydtype, nullptr, ws, st);
     return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
   }
-  // prepare the shared input once, then run every member on it
+  // prepare the shared input once, then run the members on it (one launch
+  // over all members' rows when they all use the CUDA-core decode kernel)
   size_t lin = 0;
   for (int g = 0; g < G; ++g)
     lin = std::max(lin, phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w[g]) : prefill_ws_bytes(M, w[g]));
@@ -228,6 +235,14 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   int8_t* xq = reinterpret_cast<int8_t*>(base + align256(lin));
   float* sx = reinterpret_cast<float*>(base + align256(lin) + align256((size_t)M * K));
   e = launch_quant_act(x, M, K, ldx, xq, sx, st);
+  bool rows_all = phase == AQ_PHASE_DECODE;
+  for (int g = 0; g < G; ++g) rows_all = rows_all && plan_decode(M, w[g]).kernel == 0;
+  if (e == cudaSuccess && rows_all) {  // one CUDA-core launch over all members' rows
+    DecodeProj d[kMaxGroup];
+    for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
+    e = launch_decode_rows(d, G, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+    return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+  }
   for (int g = 0; e == cudaSuccess && g < G; ++g) {
     const float* b = bias ? bias[g] : nullptr;
     if (phase == AQ_PHASE_DECODE && plan_decode(M, w[g]).kernel == 0) {

@@ -377,8 +377,6 @@ cudaError_t launch_rows_m(const RowsArgs& a, int blocks, size_t smem, cudaStream
 
 bool rows_supported(int M, int K) { return M >= 1 && M <= kRowsMaxM && K / kTileK <= kMaxC; }
 
-bool rows_fusable(int M, int K) { return 2 * (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
-
 cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
                                const float* sx, int M, int ydtype, int32_t* P, void* /*ws*/, cudaStream_t st) {
   RowsArgs a;
