@@ -20,6 +20,7 @@ int validate_packed(const aq_packed* w) {
 }
 
 static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+static constexpr int kMaxSplits = 8;
 
 // Fusing the activation preparation into every CTA of the CUDA-core decode
 // kernel pays off for 1-2 tokens; from 4 tokens on, one preparation kernel plus
@@ -27,9 +28,9 @@ static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 // preparation grows with M).  The fused codes live in shared memory.
 bool rows_fusable(int M, int K) { return M <= 2 && 2 * (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
 
-// Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, one CTA per 16
+// Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, one CTA per 32
 // output rows, no split); more tokens on the tensor cores with splits over
-// tile columns to fill the GPU.
+// tile columns to fill the GPU in one wave.
 DecodePlan plan_decode(int M, const aq_packed* w) {
   DecodePlan p;
   if (rows_supported(M, w->K)) {
@@ -41,7 +42,9 @@ DecodePlan plan_decode(int M, const aq_packed* w) {
     p.kernel = 1;
     p.rows = 128;
     p.blocks = ceil_div(w->R, 128 / w->bN);
-    p.S = std::max(1, std::min(w->C, ceil_div(kNumSMs, p.blocks)));
+    // one wave (blocks x S <= SMs), and at most kMaxSplits: the CTA that sums a
+    // unit's splits pays one round of L2 latency per split
+    p.S = std::max(1, std::min(std::min(w->C, kMaxSplits), kNumSMs / p.blocks));
   }
   return p;
 }

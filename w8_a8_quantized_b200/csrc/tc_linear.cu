@@ -662,12 +662,21 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       if (*last_flag) {
         __threadfence();
         if (rvalid) {
+          // splits outer, columns inner: the kCols loads of a split are independent
+          // and all in flight together (split order stays increasing)
+          float sum[kCols];
+#pragma unroll
+          for (int i = 0; i < kCols; ++i) sum[i] = 0.f;
+          for (int ss = 0; ss < a.S; ++ss) {
+            const float* ps = a.partial + (size_t)ss * a.M * a.N + n;
+#pragma unroll
+            for (int i = 0; i < kCols; ++i)
+              if (mcol0 + i < a.M) sum[i] += __ldcg(ps + (size_t)(mcol0 + i) * a.N);
+          }
+#pragma unroll
           for (int i = 0; i < kCols; ++i) {
             const int m = mcol0 + i;
-            if (m >= a.M) break;
-            float sum = 0.f;
-            for (int ss = 0; ss < a.S; ++ss) sum += __ldcg(a.partial + ((size_t)ss * a.M + m) * a.N + n);
-            store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sum, bias_n));
+            if (m < a.M) store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sum[i], bias_n));
           }
         }
         if (ew == 0 && lane == 0) a.counters[x.rb * a.ntb + x.tb] = 0;
