@@ -392,7 +392,9 @@ cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint
   // split the tile columns of a CTA over KG thread groups so that ~16 warps per SM stay busy
   const int warps = blocks * (kGroupThreads / 32);
   // at most 256 threads (room for the next launch's CTAs) unless rows are long
-  const int kg_cap = a.C >= 32 ? kMaxKG : 4;
+  // or the launch has no more CTAs than SMs (then wider CTAs only shorten the
+  // per-thread tile loop; with more CTAs 512-thread CTAs would need a second wave)
+  const int kg_cap = (a.C >= 32 || blocks <= kNumSMs) ? kMaxKG : 4;
   int KG = 1;
   while (KG < kg_cap && warps * KG < 16 * kNumSMs && a.C >= 4 * KG) KG *= 2;
   a.KG = KG;
