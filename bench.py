@@ -58,10 +58,10 @@ WORKLOADS = {
 # from the ncu captures summarised in profiles/, valid only while the kernel source is unchanged
 # (sha256 prefix of the source file and the shared header).
 MEASURED_TRAFFIC = {
-    # profiles/decode_rows_llama3b_1token.md: one layer's four launches read 64,740,864 B and wrote
-    # 33,536 B -> 16,193,600 B per launch (algorithmic: 16,128,638 B per launch)
+    # profiles/decode_rows_llama3b_1token.md: one layer's four launches read 64,740,608 B and wrote
+    # 23,808 B -> 16,191,104 B per launch (algorithmic: 16,128,638 B per launch)
     "decode": {"src": ("w8_a8_quantized_b200/csrc/decode_rows.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
-               "sha": "d8573e1844bd91bb", "bytes_per_launch": 16193600},
+               "sha": "3c41a89c6895f0ad", "bytes_per_launch": 16191104},
     "prefill": {"src": ("w8_a8_quantized_b200/csrc/tc_linear.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
                 "sha": None, "bytes_per_launch": None},
 }
