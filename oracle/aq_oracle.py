@@ -33,7 +33,12 @@ Readings where the paper is silent or differs from this layer's definition
   * the in-tile element order is row-major (output row, then input column)
     for both precisions; the paper permutes into a CUTLASS layout but keeps
     one order for both precisions, which is kept;
-  * the transforms U and V are the identity (the paper's seed Phi_{-1} = I).
+  * the transforms U and V are the identity (the paper's seed Phi_{-1} = I);
+  * the float-weight quantizer of App. B.2 (eq. 5-7) is applied to each output
+    row of each tile (the scale granularity of this layer) rather than to a
+    whole tile; its error sums run over the row's columns in increasing order,
+    and the selected fp64 scale is stored rounded to fp16 (the paper stores
+    FP32).
 
 Every function here is pinned by the CPU tests to values the paper prints
 (the eq. 16 worked example, Table 16's bits per weight through eq. 18), to
@@ -279,3 +284,70 @@ def linear_codes(codes, sw, xq, sx, bK, bias=None, rows=None, cols=None):
         if bias is not None:
             bias = np.asarray(bias)[cols]
     return reconstruct(tile_partials(codes, xq, bK), sx, sw, bias)
+
+
+# ---------------------------------------------------------------------------
+# Float weights -> codes and scales (App. B.2, eq. 5-7)
+# ---------------------------------------------------------------------------
+
+def q_range(b: int):
+    """App. B.2: q_min,b = -2^(b-1), q_max,b = 2^(b-1) - 1."""
+    return -(2 ** (b - 1)), 2 ** (b - 1) - 1
+
+
+def quantize_with_scale(a, s: float, b: int) -> np.ndarray:
+    """eq. 5: Q_b(A; s) = clip to [q_min, q_max] of round_even(A / s), fp64."""
+    qmin, qmax = q_range(b)
+    a = np.asarray(a, dtype=np.float64)
+    return np.clip(np.rint(a / np.float64(s)), qmin, qmax).astype(np.int64)
+
+
+def endpoint_scale(a, b: int) -> float:
+    """eq. 6: s_0 = max{ max(0, max A) / q_max, max(0, -min A) / |q_min|, 1e-12 }."""
+    qmin, qmax = q_range(b)
+    a = np.asarray(a, dtype=np.float64)
+    return max(max(0.0, float(a.max())) / qmax, max(0.0, -float(a.min())) / abs(qmin), 1e-12)
+
+
+def squared_error(a, s: float, q) -> float:
+    """||A - s Q||_F^2 summed over the elements in increasing index order."""
+    e = 0.0
+    for av, qv in zip(np.asarray(a, dtype=np.float64).ravel(), np.asarray(q).ravel()):
+        d = float(av) - float(s) * float(qv)
+        e = e + d * d
+    return e
+
+
+def search_scale(a, b: int) -> float:
+    """eq. 7: s_i = max{(1/4 + i/128) s_0, 1e-12} for i = 0..128; the scale with
+    the smallest squared reconstruction error, the earliest i on equal errors."""
+    s0 = endpoint_scale(a, b)
+    best_s, best_e = None, None
+    for i in range(129):
+        si = max((0.25 + i / 128.0) * s0, 1e-12)
+        e = squared_error(a, si, quantize_with_scale(a, si, b))
+        if best_e is None or e < best_e:
+            best_s, best_e = si, e
+    return best_s
+
+
+def quantize_weights(w, pmap: np.ndarray, bN: int, bK: int, search: bool):
+    """Float weights W[N][K] and precision labels -> (codes int8[N][K], fp16
+    scales [N][C]).  Each output row of each tile gets its own scale: the
+    endpoint scale of eq. 6, or with ``search`` the grid minimum of eq. 7; the
+    codes are eq. 5 with that fp64 scale, and the stored scale is its fp16
+    rounding.  INT4 tiles (label 1) use b = 4, INT8 tiles b = 8."""
+    w = np.asarray(w, dtype=np.float32).astype(np.float64)
+    N, K = w.shape
+    C = K // bK
+    codes = np.zeros((N, K), dtype=np.int8)
+    scales = np.zeros((N, C), dtype=np.float16)
+    for n in range(N):
+        r = n // bN
+        for j in range(C):
+            a = w[n, j * bK:(j + 1) * bK]
+            b = 4 if int(pmap[r, j]) == W4 else 8
+            s = search_scale(a, b) if search else endpoint_scale(a, b)
+            codes[n, j * bK:(j + 1) * bK] = quantize_with_scale(a, s, b).astype(np.int8)
+            scales[n, j] = np.float16(s)
+    return codes, scales

@@ -301,3 +301,122 @@ def test_synthetic_generators_shape_and_ranges():
     xv = oracle.bf16_bits_to_f64(x)
     big = (np.abs(xv) > 8).any(axis=0)
     assert 1 <= big.sum() <= 10
+
+
+# ------------------------------------------------- float-weight quantizer pins
+
+def test_weight_quant_hand_worked_endpoint_int4():
+    # eq. 6 with b = 4: max(0.5 / 7, 1.0 / 8) = 0.125; eq. 5: 0.5/0.125 = 4,
+    # -1/0.125 = -8 (q_min reached, not clipped), 0.25/0.125 = 2
+    a = np.array([0.5, -1.0, 0.25, 0.0])
+    assert oracle.endpoint_scale(a, 4) == 0.125
+    assert list(oracle.quantize_with_scale(a, 0.125, 4)) == [4, -8, 2, 0]
+
+
+def test_weight_quant_hand_worked_endpoint_int8():
+    # b = 8: max(1.27 / 127, 0.5 / 128) = 0.01 -> codes 127, -50, 0.5 -> 0 (tie to even)
+    a = np.array([1.27, -0.5, 0.005, 0.015])
+    s = oracle.endpoint_scale(a, 8)
+    assert abs(s - 0.01) < 1e-17
+    assert list(oracle.quantize_with_scale(a, 0.01, 8)) == [127, -50, 0, 2]
+    # negative-only row: max(0, max A) = 0, so s = 2.56 / 128 and -2.56 -> -128
+    a = np.array([-2.56, -1.0])
+    assert oracle.endpoint_scale(a, 8) == 2.56 / 128
+    assert list(oracle.quantize_with_scale(a, 2.56 / 128, 8)) == [-128, -50]
+
+
+def test_weight_quant_clips_and_ties_even():
+    # scale 1: 2.5 -> 2, 3.5 -> 4, -2.5 -> -2; 9 -> 7 and -9.4 -> -8 clip at the 4-bit range
+    a = np.array([2.5, 3.5, -2.5, 9.0, -9.4])
+    assert list(oracle.quantize_with_scale(a, 1.0, 4)) == [2, 4, -2, 7, -8]
+
+
+def test_weight_quant_zero_row_floor_and_fp16_underflow():
+    w = np.zeros((2, 128), np.float32)
+    pmap = np.array([[1]], np.uint8)
+    for search in (False, True):
+        codes, scales = oracle.quantize_weights(w, pmap, 2, 128, search)
+        assert not codes.any()
+        assert np.all(scales == 0)  # 1e-12 underflows fp16 to +0
+    assert oracle.search_scale(np.zeros(4), 8) == 1e-12
+
+
+def test_weight_search_recovers_grid_row_exactly():
+    # A = s q with q reaching both 4-bit ends: every smaller grid scale clips 7,
+    # so the first zero-error scale is i = 96, (1/4 + 96/128) s0 = s0 = s.
+    q = np.array([7, -8, 1, 0, 3, -5])
+    s = 0.0390625
+    assert oracle.search_scale(q * s, 4) == s
+
+
+def test_weight_search_matches_code_brute_force():
+    # For each grid scale, minimise the error over ALL code vectors in range
+    # (no rounding rule used), then over the grid with earliest-index ties; the
+    # oracle's search must reach the same scale and error.
+    rng = np.random.default_rng(7)
+    for b in (4, 3):
+        lo, hi = -(2 ** (b - 1)), 2 ** (b - 1) - 1
+        grid = np.arange(lo, hi + 1, dtype=np.float64)
+        for trial in range(6):
+            a = rng.standard_normal(3) * (0.1 if trial % 2 else 3.0)
+            if trial == 5:
+                a[0] = 40.0 * abs(a[1])  # one large element: search shrinks the scale
+            amax = max(max(0.0, a.max()) / hi, max(0.0, -a.min()) / -lo, 1e-12)
+            best = None
+            for i in range(129):
+                si = max((0.25 + i / 128.0) * amax, 1e-12)
+                e = 0.0
+                for v in a:  # each element independently: min over the code alphabet
+                    e += float(np.min((v - si * grid) ** 2))
+                if best is None or e < best[1] - 1e-15 * max(1.0, best[1]):
+                    best = (si, e)
+            s = oracle.search_scale(a, b)
+            e = oracle.squared_error(a, s, oracle.quantize_with_scale(a, s, b))
+            assert abs(e - best[1]) <= 1e-12 * max(1.0, best[1])
+            assert oracle.squared_error(a, s, oracle.quantize_with_scale(a, s, b)) <= \
+                oracle.squared_error(a, amax, oracle.quantize_with_scale(a, amax, b))
+
+
+def test_weight_search_shrinks_scale_for_an_outlier_row():
+    # 0.9 and twenty values of 0.1: with s0 = 0.9/7 the small values round to 1
+    # (0.1/0.1286 = 0.78), each off by 0.0286; a smaller scale must win.
+    a = np.array([0.9] + [0.1] * 20)
+    s0 = oracle.endpoint_scale(a, 4)
+    s = oracle.search_scale(a, 4)
+    assert s < s0
+    e = lambda t: oracle.squared_error(a, t, oracle.quantize_with_scale(a, t, 4))
+    assert e(s) < e(s0)
+
+
+def test_quantize_weights_layout_bits_and_bound():
+    N, K, bN, bK = 8, 256, 4, 128
+    w = synth.float_weights(N, K, (11,), outlier_frac=0.01)
+    pmap = np.array([[1, 0], [0, 1]], np.uint8)
+    codes, scales = oracle.quantize_weights(w, pmap, bN, bK, search=False)
+    assert codes.shape == (N, K) and scales.shape == (N, 2) and scales.dtype == np.float16
+    wv = w.astype(np.float64)
+    for n in range(N):
+        for j in range(2):
+            a = wv[n, j * bK:(j + 1) * bK]
+            b = 4 if pmap[n // bN, j] == 1 else 8
+            c = codes[n, j * bK:(j + 1) * bK].astype(int)
+            assert c.min() >= -(2 ** (b - 1)) and c.max() <= 2 ** (b - 1) - 1
+            # the endpoint scale never clips: every element within half a step
+            s = max(a.max() / (2 ** (b - 1) - 1), -a.min() / 2 ** (b - 1))
+            assert np.abs(a - s * c).max() <= s / 2 * (1 + 1e-12)
+            assert scales[n, j] == np.float16(s)
+            # the largest magnitude reaches a range end
+            assert c.max() == 2 ** (b - 1) - 1 or c.min() == -(2 ** (b - 1))
+    # the codes pack: INT4 tiles stay within 4 bits
+    oracle.pack(codes, scales, pmap, bN, bK)
+    # search never does worse than the endpoint, row by row
+    codes_s, scales_s = oracle.quantize_weights(w[:2], pmap[:1], 2, bK, search=True)
+    for n in range(2):
+        for j in range(2):
+            a = wv[n, j * bK:(j + 1) * bK]
+            b = 4 if pmap[0, j] == 1 else 8
+            s = oracle.search_scale(a, b)
+            c = codes_s[n, j * bK:(j + 1) * bK]
+            assert np.array_equal(c, oracle.quantize_with_scale(a, s, b))
+            assert oracle.squared_error(a, s, c) <= \
+                oracle.squared_error(a, oracle.endpoint_scale(a, b), codes[n, j * bK:(j + 1) * bK])

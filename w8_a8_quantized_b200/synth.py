@@ -12,6 +12,9 @@ What it produces, per projection (N output features x K input features):
     INT8 tiles and over [-8, 7] in INT4 tiles;
   * per-row-per-tile weight scales ``scales[N][C]`` drawn uniform in
     [1e-3, 1e-2] and rounded to fp16;
+  * float weights ``W[N][K]`` (fp32) drawn N(0, 0.02^2), optionally with a
+    seeded fraction of entries multiplied by 10 (outlier weights), for the
+    weight quantizer;
   * activations ``X[M][K]`` drawn N(0, 1) in fp32, optionally with a seeded
     set of outlier input channels multiplied by 20, rounded to bf16 and
     returned as raw bf16 bit patterns (uint16).
@@ -29,6 +32,7 @@ import numpy as np
 __all__ = [
     "MODELS", "projections", "precision_map", "weight_codes", "weight_scales",
     "activations", "f32_to_bf16_bits", "projection_inputs", "SingleProjection",
+    "float_weights",
 ]
 
 # (hidden, q-proj out, k/v-proj out, MLP intermediate, layers)
@@ -100,6 +104,18 @@ def activations(M: int, K: int, seed, outlier_frac: float = 0.0, outlier_mult: f
         cols = g.choice(K, size=n_out, replace=False)
         x[:, cols] *= np.float32(outlier_mult)
     return f32_to_bf16_bits(x)
+
+
+def float_weights(N: int, K: int, seed, outlier_frac: float = 0.0, outlier_mult: float = 10.0) -> np.ndarray:
+    """float32[N][K] drawn N(0, 0.02^2); round(outlier_frac*N*K) seeded entries
+    are multiplied by outlier_mult."""
+    g = _rng(*_key(seed), 5)
+    w = (g.standard_normal((N, K), dtype=np.float32) * np.float32(0.02))
+    n_out = int(round(outlier_frac * N * K))
+    if n_out:
+        idx = g.choice(N * K, size=n_out, replace=False)
+        w.reshape(-1)[idx] *= np.float32(outlier_mult)
+    return w
 
 
 def _key(seed):
