@@ -42,7 +42,7 @@ typedef enum {
   AQ_OK = 0,
   AQ_ERR_ARG = -1,         /* null pointer, bad enum, misaligned pointer, M/K/ld out of range */
   AQ_ERR_SHAPE = -2,       /* N, K, bN, bK violate the tile geometry */
-  AQ_ERR_RANGE = -3,       /* an INT4 tile holds a code outside [-8, 7] (aq_pack) */
+  AQ_ERR_RANGE = -3,       /* an INT4 code outside [-8, 7] (aq_pack); a non-finite weight (aq_quantize_weights) */
   AQ_ERR_UNSUPPORTED = -4, /* a valid request this build does not implement */
   AQ_ERR_WORKSPACE = -5,   /* workspace missing or smaller than aq_workspace_bytes() */
   AQ_ERR_CUDA = -6,        /* a CUDA runtime call or a kernel launch failed */
@@ -105,6 +105,20 @@ const char* aq_status_str(int status);
 int aq_packed_sizes(int N, int K, int bN, int bK, int T4, size_t* out_bytes);
 
 /*
+ * Host only, no CUDA call.  Storage of a packed projection as the paper
+ * accounts it (eq. 18, App. E.2): payloads B*T4/2 + B*T8 with B = bN*bK, one
+ * 4-byte scale per tile, ceil(R*C/8) label bytes and two (R+1)-entry 4-byte
+ * row-offset arrays; T8 = R*C - T4.  Summing it over a model's quantized
+ * projections, times 8, over their weight count gives the packed bits per
+ * weight of App. G.7 / Table 16.  Any tile shape (bN, bK >= 1, bN*bK even) is
+ * accepted; this is accounting only and differs from aq_packed_sizes (fp16
+ * scale per row per tile, plus the physical-index table).
+ * Errors: AQ_ERR_ARG (null out_bytes, R, C, bN or bK < 1, odd bN*bK, T4 outside
+ * [0, R*C]).
+ */
+int aq_paper_packed_bytes(int R, int C, int T4, int bN, int bK, size_t* out_bytes);
+
+/*
  * Host only, no CUDA call.  Metadata of the packed format from a HOST copy of
  * the precision labels map[R][C] (1 = INT4, 0 = INT8): bitmap, both row-offset
  * arrays and tile_idx, written to HOST buffers of the sizes aq_packed_sizes()
@@ -130,6 +144,31 @@ int aq_pack_metadata(const uint8_t* map_host, int R, int C, uint8_t* bitmap, int
  */
 int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_t* map, int N, int K, int bN,
             int bK, aq_packed* out, void* stream);
+
+/*
+ * Float weights -> integer codes and scales for aq_pack (App. B.2, eq. 5-7),
+ * one scale per output row per tile.  For row n of tile (r, j), A = the bK
+ * values w[n][j*bK .. j*bK+bK-1] and b = 4 (INT4 label) or 8 (INT8 label):
+ *   s0 = max(max(0, max A) / (2^(b-1) - 1), max(0, -min A) / 2^(b-1), 1e-12)   (eq. 6)
+ *   search == 0: s* = s0
+ *   search == 1: s* = the s_i = max((1/4 + i/128) s0, 1e-12), i = 0..128, with
+ *                the least sum_k (A_k - s_i Q_k)^2, earliest i on ties      (eq. 7)
+ *   codes[n][k] = clip(rint(A_k / s*), -2^(b-1), 2^(b-1) - 1)            (eq. 5)
+ *   scales[n][j] = fp16(s*), rounded to nearest even from fp64
+ * in fp64, each operation rounded separately, error sums in increasing k.
+ *  w      fp32 or bf16 (wdtype, aq_dtype) [N][ldw] device, 16-byte aligned,
+ *         ldw >= K, ldw % 4 == 0 (fp32) or ldw % 8 == 0 (bf16); read only
+ *  map    uint8 [R][C] device, 1 = INT4 tile, 0 = INT8 tile
+ *  codes  int8  [N][K] device, 16-byte aligned (written)
+ *  scales fp16  [N][C] device, bits as uint16 (written)
+ * Offline step: synchronizes `stream` and allocates a few bytes of temporary
+ * device memory.  Errors: AQ_ERR_ARG (null or misaligned pointer, bad wdtype
+ * or search, ldw out of range, a label other than 0 or 1), AQ_ERR_SHAPE,
+ * AQ_ERR_RANGE (a weight is NaN or infinite; outputs then unspecified),
+ * AQ_ERR_CUDA.
+ */
+int aq_quantize_weights(const void* w, int wdtype, int N, int K, int ldw, int bN, int bK, const uint8_t* map,
+                        int search, int8_t* codes, uint16_t* scales, void* stream);
 
 /*
  * Per-token symmetric INT8 quantization of activations (App. B.3 computed per

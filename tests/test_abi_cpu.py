@@ -118,6 +118,18 @@ def test_host_validation_rejects_before_any_launch():
                             bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=18)
     assert L.aq_linear_prefill(ctypes.byref(mis), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
     assert L.aq_linear_decode(ctypes.byref(mis), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    # weight quantizer: null, dtype, search flag, geometry, ldw and alignment
+    qw = L.aq_quantize_weights
+    assert qw(None, 0, 128, 128, 128, 128, 128, 16, 1, 16, 16, None) == -1
+    assert qw(16, 2, 128, 128, 128, 128, 128, 16, 1, 16, 16, None) == -1
+    assert qw(16, 0, 128, 128, 128, 128, 128, 16, 2, 16, 16, None) == -1
+    assert qw(16, 0, 100, 128, 128, 128, 128, 16, 1, 16, 16, None) == -2
+    assert qw(16, 0, 128, 128, 128, 128, 64, 16, 1, 16, 16, None) == -2
+    assert qw(16, 0, 128, 128, 120, 128, 128, 16, 1, 16, 16, None) == -1
+    assert qw(16, 0, 128, 128, 130, 128, 128, 16, 1, 16, 16, None) == -1
+    assert qw(16, 1, 128, 128, 132, 128, 128, 16, 1, 16, 16, None) == -1
+    assert qw(20, 0, 128, 128, 128, 128, 128, 16, 1, 16, 16, None) == -1
+    assert qw(16, 0, 128, 128, 128, 128, 128, 16, 1, 24, 16, None) == -1
     assert L.aq_workspace_bytes(0, 65, ctypes.byref(s)) == 0
     assert L.aq_workspace_bytes(0, 1, ctypes.byref(s)) >= 256
     assert L.aq_workspace_bytes(5, 1, ctypes.byref(s)) == 0
@@ -154,3 +166,35 @@ def test_group_workspace_sizes():
     bad.K, bad.C = 2048, 16
     arr2 = (P * 2)(ctypes.pointer(q), ctypes.pointer(bad))
     assert L.aq_group_workspace_bytes(0, 1, arr2, 2) == 0
+
+
+def test_paper_accounting_reproduces_table16():
+    # App. H.3.3 Table 16 packed bits per weight for the Llama-3.2-3B shapes at
+    # 64 x 64 tiles, model-wide W4 count round(rho |T|) filled projection by
+    # projection, through the library's eq. 18 accounting
+    import json, os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "table16_packed_bpw.json")) as f:
+        g = json.load(f)
+    bN, bK = g["tile"]
+    shapes = synth.projections("llama-3.2-3b") * synth.MODELS["llama-3.2-3b"]["layers"]
+    tiles = [(n // bN) * (k // bK) for _, n, k in shapes]
+    for rho, want in zip(g["w4_fraction"], g["packed_bpw_2dp"]):
+        left, S, W = int(round(rho * sum(tiles))), 0, 0
+        for (_, n, k), t in zip(shapes, tiles):
+            t4 = min(left, t)
+            left -= t4
+            S += aq.aq_paper_packed_bytes(n // bN, k // bK, t4, bN, bK)
+            W += n * k
+        assert round(8 * S / W, 2) == pytest.approx(want, abs=1e-9), rho
+
+
+@pytest.mark.parametrize("R,C,T4,bN,bK", [(1, 1, 0, 2, 2), (3, 5, 7, 64, 64), (40, 24, 960, 128, 128),
+                                          (17, 9, 0, 64, 128), (2, 3, 6, 1, 2)])
+def test_paper_accounting_matches_oracle_and_rejects(R, C, T4, bN, bK):
+    assert aq.aq_paper_packed_bytes(R, C, T4, bN, bK) == oracle.paper_packed_bytes(R, C, T4, bN, bK)
+    L, out = aq.lib(), ctypes.c_size_t()
+    assert L.aq_paper_packed_bytes(R, C, R * C + 1, bN, bK, ctypes.byref(out)) == -1
+    assert L.aq_paper_packed_bytes(R, C, -1, bN, bK, ctypes.byref(out)) == -1
+    assert L.aq_paper_packed_bytes(R, C, T4, 3, 3, ctypes.byref(out)) == -1
+    assert L.aq_paper_packed_bytes(0, C, 0, bN, bK, ctypes.byref(out)) == -1
+    assert L.aq_paper_packed_bytes(R, C, T4, bN, bK, None) == -1

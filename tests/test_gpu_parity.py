@@ -4,6 +4,8 @@ Integer and byte results (packed buffers, activation codes and scales, per-tile
 INT32 products) must be bit-exact.  Floating-point outputs must meet the
 tolerance in aq_testutil.assert_output_close.  Sizes span several tiles with
 ragged token counts and, for 64-row tiles, an odd number of tile rows."""
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -274,3 +276,124 @@ def test_quant_act_every_bf16_absmax():
     xq_ref, sx_ref = oracle.quant_act(x)
     assert np.array_equal(sx.cpu().numpy().view(np.uint32), sx_ref.view(np.uint32))
     assert np.array_equal(xq.cpu().numpy(), xq_ref)
+
+
+# ------------------------------------------------------------------ float-weight quantizer
+
+def _crafted_weights(N, K, seed):
+    """Random weights with rows that reach the method's special cases."""
+    w = synth.float_weights(N, K, (seed,), outlier_frac=0.002)
+    rng = np.random.default_rng(seed)
+    w[0, 0:128] = 0.0                                                    # zero row: scale floor, fp16 0
+    w[1, 0:128] = -np.abs(w[1, 0:128])                                   # negative-only row
+    # quarter steps of s0 = 0.125 (INT4 tile): A / s_i hits exact half-integers at i = 32 and 96
+    w[2, 0:128] = (rng.integers(-32, 29, 128) / 4.0 * 0.125).astype(np.float32)
+    w[2, 0], w[2, 1] = 7 * 0.125, -8 * 0.125
+    w[3, 0:128] = (rng.standard_normal(128) * 1e-6).astype(np.float32)  # fp16 subnormal scales
+    w[4, 0:128] = 0.01
+    w[4, 5] = 7.0 * (1 + 2.0 ** -11)                                     # s0 = 1 + 2^-11: fp16 tie -> 1.0
+    w[5, 0:128] = 0.02
+    w[5, 9] = 7.0 * (1 + 3 * 2.0 ** -11)                                 # fp16 tie -> 1 + 2^-9
+    w[6, 0:128] = 0.1
+    w[6, 0] = 0.9                                                        # the search shrinks the scale
+    w[7, 128:256] = 3.0e6                                                # scale beyond fp16: infinity
+    return w
+
+
+def _oracle_quantize(w, pmap, bN, search):
+    with np.errstate(over="ignore"):
+        return oracle.quantize_weights(w, pmap, bN, 128, search)
+
+
+@pytest.mark.parametrize("search", [False, True])
+@pytest.mark.parametrize("bN,wdtype", [(64, torch.float32), (128, torch.bfloat16)])
+def test_quantize_weights_bit_exact(search, bN, wdtype):
+    N, K = 128, 384
+    w = _crafted_weights(N, K, 21)
+    pmap = synth.precision_map(N // bN, K // 128, 0.5, (22,))
+    pmap[0, 0] = 1
+    pmap[0, 1] = 1
+    if wdtype == torch.bfloat16:
+        bits = synth.f32_to_bf16_bits(w)
+        w = oracle.bf16_bits_to_f64(bits).astype(np.float32)
+        wd = dev_bf16(bits)
+    else:
+        wd = torch.from_numpy(w).cuda()
+    codes, scales = aq.aq_quantize_weights(wd, torch.from_numpy(pmap).cuda(), bN, 128, search)
+    rc, rs = _oracle_quantize(w, pmap, bN, search)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
+
+
+def test_quantize_weights_strided_input_and_all_int8():
+    N, K, ldw = 64, 256, 384
+    big = synth.float_weights(N, ldw, (31,), outlier_frac=0.01)
+    pmap = np.zeros((1, 2), np.uint8)
+    wd = torch.from_numpy(big).cuda()[:, :K]
+    codes, scales = aq.aq_quantize_weights(wd, torch.from_numpy(pmap).cuda(), 64, 128, True)
+    rc, rs = _oracle_quantize(np.ascontiguousarray(big[:, :K]), pmap, 64, True)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), rs.view(np.uint16))
+
+
+@pytest.mark.parametrize("search", [False, True])
+def test_quantize_weights_full_size_sampled(search):
+    # a 4096 x 4096 projection with 128-row tiles; the oracle checks 40 sampled
+    # (row, tile) pairs one by one, every code is checked against its range
+    N = K = 4096
+    w = synth.float_weights(N, K, (41,), outlier_frac=0.001)
+    pmap = synth.precision_map(N // 128, K // 128, 0.25, (42,))
+    codes, scales = aq.aq_quantize_weights(torch.from_numpy(w).cuda(), torch.from_numpy(pmap).cuda(), 128, 128,
+                                           search)
+    codes, scales = codes.cpu().numpy(), scales.cpu().numpy()
+    is4 = np.repeat(np.repeat(pmap.astype(bool), 128, 0), 128, 1)
+    assert codes[is4].min() >= -8 and codes[is4].max() <= 7
+    rng = np.random.default_rng(43)
+    for n, j in zip(rng.integers(0, N, 40), rng.integers(0, K // 128, 40)):
+        seg = w[n:n + 1, j * 128:(j + 1) * 128]
+        rc, rs = _oracle_quantize(seg, pmap[n // 128:n // 128 + 1, j:j + 1], 1, search)
+        assert np.array_equal(codes[n, j * 128:(j + 1) * 128], rc[0])
+        assert scales[n, j].view(np.uint16) == rs[0, 0].view(np.uint16)
+
+
+def test_quantize_weights_reports_non_finite():
+    w = synth.float_weights(64, 128, (51,))
+    w[10, 17] = np.nan
+    pmap = torch.ones((1, 1), dtype=torch.uint8, device="cuda")
+    with pytest.raises(aq.AqError) as e:
+        aq.aq_quantize_weights(torch.from_numpy(w).cuda(), pmap, 64, 128, True)
+    assert e.value.status == -3
+    w[10, 17] = np.inf
+    with pytest.raises(aq.AqError) as e:
+        aq.aq_quantize_weights(torch.from_numpy(w).cuda(), pmap, 64, 128, False)
+    assert e.value.status == -3
+    with pytest.raises(aq.AqError) as e:  # a label other than 0 / 1
+        aq.aq_quantize_weights(torch.zeros((64, 128), device="cuda"), pmap * 2, 64, 128, False)
+    assert e.value.status == -1
+
+
+_QP = dict(N=256, K=512, bN=128)
+
+
+@functools.lru_cache(maxsize=1)
+def _quantize_and_pack_case():
+    N, K, bN = _QP["N"], _QP["K"], _QP["bN"]
+    w = synth.float_weights(N, K, (61,), outlier_frac=0.005)
+    pmap = synth.precision_map(N // bN, K // 128, 0.5, (62,))
+    return w, pmap, _oracle_quantize(w, pmap, bN, True)
+
+
+@pytest.mark.parametrize("M", [1, 8, 300])
+def test_quantize_and_pack_feeds_the_linear_layer(M):
+    N, K, bN = _QP["N"], _QP["K"], _QP["bN"]
+    w, pmap, (rc, rs) = _quantize_and_pack_case()
+    pw = aq.aq_quantize_and_pack(torch.from_numpy(w).cuda(), torch.from_numpy(pmap).cuda(), bN, 128, True)
+    ref = oracle.pack(rc, rs, pmap, bN, 128)
+    got = pw.host_buffers()
+    for name in aq.BUF_NAMES:
+        assert np.array_equal(got[name], np.ascontiguousarray(ref[name]).view(np.uint8).reshape(-1)), name
+    x = synth.activations(M, K, (63, M))
+    xq, sx = aq.aq_quant_act(dev_bf16(x))
+    y = (aq.aq_linear_decode if M <= 64 else aq.aq_linear_prefill)(pw, xq, sx)
+    ref_p = synth.SingleProjection(N, K, bN, 128, pmap, rc, rs)
+    assert_output_close(y, oracle_linear(ref_p, x))

@@ -21,7 +21,8 @@ AQ_PHASE_DECODE, AQ_PHASE_PREFILL = 0, 1
 BUF_NAMES = ("bitmap", "row_off4", "row_off8", "tile_idx", "w4", "w8", "scales")
 EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "aq_quant_act",
             "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
-            "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc")
+            "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc",
+            "aq_quantize_weights", "aq_paper_packed_bytes")
 
 
 class AqError(RuntimeError):
@@ -59,6 +60,11 @@ def lib():
     L.aq_pack.restype = c_int
     L.aq_pack.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, P, c_void_p]
     L.aq_quant_act.restype = c_int
+    L.aq_paper_packed_bytes.restype = c_int
+    L.aq_paper_packed_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_size_t)]
+    L.aq_quantize_weights.restype = c_int
+    L.aq_quantize_weights.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_int,
+                                      c_void_p, c_void_p, c_void_p]
     L.aq_quant_act.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
     L.aq_workspace_bytes.restype = c_size_t
     L.aq_workspace_bytes.argtypes = [c_int, c_int, P]
@@ -108,6 +114,13 @@ def aq_packed_sizes(N: int, K: int, bN: int, bK: int, T4: int) -> dict:
     return dict(zip(BUF_NAMES, [int(v) for v in out]))
 
 
+def aq_paper_packed_bytes(R: int, C: int, T4: int, bN: int, bK: int) -> int:
+    """Storage of one packed projection as eq. 18 accounts it (FP32 scale per tile)."""
+    out = ctypes.c_size_t()
+    _check(lib().aq_paper_packed_bytes(R, C, T4, bN, bK, ctypes.byref(out)), "aq_paper_packed_bytes")
+    return int(out.value)
+
+
 class PackedWeights:
     """Device buffers of one packed projection plus the C struct describing them."""
 
@@ -150,6 +163,37 @@ def aq_pack(codes: torch.Tensor, scales: torch.Tensor, pmap: torch.Tensor, bN: i
     _check(lib().aq_pack(codes.data_ptr(), scales.data_ptr(), pmap.data_ptr(), N, K, bN, bK,
                          ctypes.byref(w.struct), _stream(dev)), "aq_pack")
     return w
+
+
+def aq_quantize_weights(w: torch.Tensor, pmap: torch.Tensor, bN: int, bK: int = 128, search: bool = True,
+                        codes: torch.Tensor = None, scales: torch.Tensor = None):
+    """Float weights w (float32 or bfloat16, [N][ldw] with unit inner stride) and
+    labels pmap uint8 [R][C] (1 = INT4) -> (codes int8 [N][K], scales float16
+    [N][C]) for aq_pack.  K = pmap.shape[1] * bK; search selects eq. 7's scale
+    search over eq. 6's endpoint scale."""
+    if w.dim() != 2 or not w.is_cuda or w.stride(1) != 1 or w.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("w must be a 2-D float32 or bfloat16 CUDA tensor with unit inner stride")
+    dev = w.device
+    _need(pmap, "pmap", torch.uint8, dev)
+    N, K = w.shape[0], pmap.shape[1] * bK
+    if codes is None:
+        codes = torch.empty((N, K), dtype=torch.int8, device=dev)
+    if scales is None:
+        scales = torch.empty((N, pmap.shape[1]), dtype=torch.float16, device=dev)
+    _need(codes, "codes", torch.int8, dev)
+    _need(scales, "scales", torch.float16, dev)
+    wdtype = AQ_F32 if w.dtype == torch.float32 else AQ_BF16
+    _check(lib().aq_quantize_weights(w.data_ptr(), wdtype, N, K, w.stride(0), bN, bK, pmap.data_ptr(),
+                                     int(bool(search)), codes.data_ptr(), scales.data_ptr(), _stream(dev)),
+           "aq_quantize_weights")
+    return codes, scales
+
+
+def aq_quantize_and_pack(w: torch.Tensor, pmap: torch.Tensor, bN: int, bK: int = 128,
+                         search: bool = True) -> PackedWeights:
+    """Float weights -> packed tile format: aq_quantize_weights then aq_pack."""
+    codes, scales = aq_quantize_weights(w, pmap, bN, bK, search)
+    return aq_pack(codes, scales, pmap, bN, bK)
 
 
 def aq_quant_act(x: torch.Tensor, xq: torch.Tensor = None, sx: torch.Tensor = None, K: int = None):

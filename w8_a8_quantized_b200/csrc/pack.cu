@@ -99,6 +99,16 @@ extern "C" int aq_pack_metadata(const uint8_t* map_host, int R, int C, uint8_t* 
   return AQ_OK;
 }
 
+extern "C" int aq_paper_packed_bytes(int R, int C, int T4, int bN, int bK, size_t* out_bytes) {
+  if (!out_bytes || R < 1 || C < 1 || bN < 1 || bK < 1) return AQ_ERR_ARG;
+  const unsigned long long B = (unsigned long long)bN * bK, T = (unsigned long long)R * C;
+  if ((B & 1) || T4 < 0 || (unsigned long long)T4 > T) return AQ_ERR_ARG;
+  const unsigned long long T8 = T - (unsigned long long)T4;
+  // eq. 18: payloads, one FP32 scale per tile, labels, two row-offset arrays
+  *out_bytes = (size_t)(B * T4 / 2 + B * T8 + 4 * T + (T + 7) / 8 + 8 * ((unsigned long long)R + 1));
+  return AQ_OK;
+}
+
 extern "C" int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_t* map, int N, int K, int bN,
                        int bK, aq_packed* out, void* stream) {
   using namespace aq;
