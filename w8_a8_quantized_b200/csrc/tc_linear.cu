@@ -23,30 +23,32 @@
 //   warp 3      activation producer: the NT x 128 INT8 activation tile -> B
 //               stage (TMA), after the previous kernel (which writes the
 //               activations) is done.
-//   warps 4..   epilogue; warp w may read tensor-memory lanes 32 (w % 4) ..
+//   warps 4-7   transform: one thread per row of the 128-row block.  Tile by
+//               tile they put each row's weight scale (fp16 -> fp32, / 16 for
+//               INT4) into a shared-memory ring and expand the INT4 staging
+//               tiles into the 128-byte-swizzled INT8 A layout
+//               (fence.proxy.async before signalling the MMA).  They run ahead
+//               of the epilogue, bounded only by the stage ring.
+//   warps 8..   epilogue; warp w may read tensor-memory lanes 32 (w % 4) ..
 //               32 (w % 4) + 31.  After every input tile it reads the INT32
-//               tile product from tensor memory, multiplies by the row's fp16
+//               tile product from tensor memory, multiplies by the row's
 //               weight scale of that tile and accumulates in FP32 registers;
 //               at the end of a work unit it multiplies by the token scale,
-//               adds bias and stores.
-//               The same warps expand the INT4 staging tiles into the
-//               128-byte-swizzled INT8 A layout kExpandAhead tiles ahead of
-//               the tile they rescale (fence.proxy.async before signalling the
-//               MMA), and at that point copy their row's weight scale of the
-//               tile into a private shared-memory ring, so the rescale itself
-//               waits on nothing but the accumulator.  Tiles are rescaled in
-//               pairs: one accumulator wait and one release per two tiles.
+//               adds bias and stores.  Tiles are rescaled in pairs (one
+//               accumulator wait and one release per two tiles) and the
+//               tensor-memory loads are software pipelined: the next 16
+//               columns are in flight while the current ones are rescaled.
 // A single thread on a busy SM retires roughly one dependent instruction every
 // 10-20 cycles, so the per-tile work of each issuing thread is kept to a few
-// dozen instructions and spread over three threads.
+// dozen instructions and spread over three threads, and everything the
+// epilogue does per tile besides the rescale runs in other warps.
 // Weights are the A operand, so TMEM lane = output row and each epilogue
 // thread applies ONE weight scale per input tile.
 //
 // The FP32 rescale is the co-bottleneck of this design: per input tile and
 // output element it costs one add and one fused multiply-add on the CUDA
 // cores, as many cycles per SM as the INT8 MMA itself; the float2 forms
-// halve the issue slots it takes so tensor-memory and expansion work fit
-// beside it.
+// halve the issue slots it takes so tensor-memory work fits beside it.
 //
 // A work unit is (128-row block of output features, NT-token block, split of
 // the input tiles).  Split partial sums go to the workspace; the CTA that
@@ -65,14 +67,11 @@ namespace aq {
 namespace {
 
 constexpr int kBufs = 4;        // accumulator buffers in tensor memory
-constexpr int kSwRing = 8;      // per-thread ring of expanded-ahead weight scales (> kExpandAhead + 1)
+constexpr int kSwRing = 16;     // ring of per-row weight scales, one slot per tile (> stages + kBufs)
 constexpr int kMetaSlots = 32;  // metadata ring slots (one per lane of the metadata warp)
-constexpr int kFirstEpiWarp = 4;
-// Tiles the epilogue expands ahead of the one it rescales.  At least kBufs,
-// so the MMA (at most kBufs tiles ahead of the epilogue) never waits for an
-// expansion; below stages + kBufs (counting the second tile of a pair), so the
-// staging copy it waits for never depends on the epilogue's own later progress.
-constexpr int kExpandAhead = kBufs;
+constexpr int kFirstXfWarp = 4;   // transform warps: INT4 expansion and per-row weight scales
+constexpr int kXfWarps = 4;       // 128 threads, one per row of the 128-row block
+constexpr int kFirstEpiWarp = kFirstXfWarp + kXfWarps;
 
 template <int NT>
 struct TcShape {
@@ -84,11 +83,10 @@ struct TcShape {
   static constexpr int kCols = NT <= 64 ? NT : 64;  // accumulator columns per epilogue thread
   static constexpr int kEpiWarps = 4 * NT / kCols;      // 4 warps (one per lane quadrant) per column group
   static constexpr int kThreads = 32 * kFirstEpiWarp + 32 * kEpiWarps;
-  // Tensor-memory columns per load wait: all of them up to 48; 64 columns take
-  // two waits, which keeps the loaded values and the accumulators within the
-  // register budget.
-  static constexpr int kLdCols = kCols <= 48 ? kCols : 32;
-  static_assert(kCols % kLdCols == 0 && kLdCols % 16 == 0, "load chunks");
+  // Tensor-memory columns per load (one 16-column load; two register sets are
+  // live while the loads are pipelined).
+  static constexpr int kLdCols = 16;
+  static_assert(kCols % kLdCols == 0, "load chunks");
   // Registers per thread: the register file over the block's warps, counted in
   // groups of four warps as the hardware allocates them (an explicit cap: the
   // block-size bound makes the compiler trade registers for spills here).
@@ -97,7 +95,7 @@ struct TcShape {
   static constexpr int kTmemCols = kBufs * NT <= 32 ? 32 : kBufs * NT <= 64 ? 64 : kBufs * NT <= 128 ? 128
                                    : kBufs * NT <= 256 ? 256 : 512;
   static constexpr int kScBytes = kStages * 256;  // per stage: the tile's 128 row scales (fp16)
-  static constexpr int kSwBytes = kSwRing * 32 * kEpiWarps * 4;  // [kSwRing][epilogue thread] fp32
+  static constexpr int kSwBytes = kSwRing * 128 * 4;  // [kSwRing][row] fp32
   static constexpr int kCtrlBytes = 2048;
   static constexpr int kPreBytes = (32 + kCols) * kEpiWarps * 4;  // per-unit bias and token scales of the epilogue
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kScBytes + kCtrlBytes + kPreBytes + kSwBytes;
@@ -106,10 +104,10 @@ struct TcShape {
   static_assert(kBufs * NT <= 512, "tensor memory");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kStages >= 3, "ring depth");
-  // pairs of tiles: the epilogue expands up to tile g + 1 + kExpandAhead while
-  // it still holds tile g
-  static_assert(kExpandAhead >= kBufs && kExpandAhead + 1 < kStages + kBufs, "expansion distance");
-  static_assert(kSwRing > kExpandAhead + 1, "scale ring depth");
+  // the transform warps run at most kStages + kBufs tiles ahead of the epilogue
+  // (a stage is refilled only after its MMAs, which wait for an accumulator
+  // buffer the epilogue released), so a scale slot is never rewritten early
+  static_assert(kStages + kBufs < kSwRing, "scale ring depth");
   static_assert(kThreads <= 1024, "block size");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -267,7 +265,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
   uint8_t* ctrl = stage_sc + Sh::kScBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);  // weights (INT8) + activations landed; one arrival per producer
   uint64_t* staged = full + S_;                        // INT4 staging landed (0 bytes when none)
-  uint64_t* expanded = staged + S_;                    // epilogue warps done expanding the stage (one arrival each)
+  uint64_t* expanded = staged + S_;                    // transform warps done with the stage (one arrival each)
   uint64_t* empty = expanded + S_;                     // MMAs reading the stage done
   uint64_t* tmem_full = empty + S_;
   uint64_t* tmem_empty = tmem_full + kBufs;
@@ -275,7 +273,8 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
   uint64_t* meta_empty = meta_full + kMetaSlots;
   uint64_t* epi_sync = meta_empty + kMetaSlots;  // epilogue-only rendezvous (bounded, unlike bar.sync)
   uint64_t* drain = epi_sync + 1;                // MMA completion on the way out
-  MetaRec* meta = reinterpret_cast<MetaRec*>(drain + 1);
+  uint64_t* sw_full = drain + 1;                 // [kSwRing] scale slot written (one arrival per transform warp)
+  MetaRec* meta = reinterpret_cast<MetaRec*>(sw_full + kSwRing);
   volatile uint32_t* stage_info = reinterpret_cast<volatile uint32_t*>(meta + kMetaSlots);
   uint32_t* tmem_slot = const_cast<uint32_t*>(stage_info + S_);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -283,8 +282,8 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
   volatile int* never_flag = reinterpret_cast<volatile int*>(tmem_slot + 3);  // stays 0: drain waits
   float* pre_bias = reinterpret_cast<float*>(ctrl + Sh::kCtrlBytes);  // [32 kEpiWarps] bias of each epilogue row
   float* pre_sx = pre_bias + 32 * Sh::kEpiWarps;                       // [kEpiWarps][kCols] token scales
-  float* pre_sw = pre_sx + Sh::kEpiWarps * Sh::kCols;                    // [kSwRing][32 kEpiWarps] weight scales
-  static_assert((4 * 8 + 2 * kBufs + 2 * kMetaSlots + 2) * 8 + kMetaSlots * 16 + (8 + 4) * 4 <=
+  float* pre_sw = pre_sx + Sh::kEpiWarps * Sh::kCols;                    // [kSwRing][128] weight scale of each row
+  static_assert((4 * 8 + 2 * kBufs + 2 * kMetaSlots + 2 + kSwRing) * 8 + kMetaSlots * 16 + (8 + 4) * 4 <=
                     Sh::kCtrlBytes,
                 "control area");
 
@@ -293,7 +292,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
     for (int st = 0; st < S_; ++st) {
       mbar_init(&full[st], 2);
       mbar_init(&staged[st], 1);
-      mbar_init(&expanded[st], Sh::kEpiWarps);
+      mbar_init(&expanded[st], kXfWarps);
       mbar_init(&empty[st], 1);
     }
     for (int b = 0; b < kBufs; ++b) {
@@ -306,6 +305,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
     }
     mbar_init(epi_sync, 32 * Sh::kEpiWarps);
     mbar_init(drain, 1);
+    for (int i = 0; i < kSwRing; ++i) mbar_init(&sw_full[i], kXfWarps);
     *abort_flag = 0;
     *never_flag = 0;
     fence_mbar_init();
@@ -342,7 +342,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(2); ok = false; break; }
         const uint32_t kinds = rec.sizes >> 28;
         const uint32_t sc_bytes = (kinds & 8) ? 4u * a.bN : 2u * a.bN;  // fp16 row scales of the tile's sub-tiles
-        stage_info[sr.i] = kinds;  // read by the expanding epilogue warps after `staged`
+        stage_info[sr.i] = kinds;  // read by the transform warps after `staged`
         mbar_arrive_expect_tx(&full[sr.i], (rec.sizes & 0xFFu) << 10);
         mbar_arrive_expect_tx(&staged[sr.i], (((rec.sizes >> 8) & 0xFFu) << 10) + sc_bytes);
         uint8_t* scd = stage_sc + sr.i * 256;
@@ -443,6 +443,51 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       }
       if (!ok || *abort_flag) abort_grace();
     }
+  } else if (warp < kFirstEpiWarp) {
+    // ------------------------------------------------------------ transform
+    // Tile by tile, in the order of the stage ring: the per-row weight scale
+    // (0 for a row past the layer's end; / 16 for INT4, whose codes are
+    // expanded as 16 q) into its ring slot, then the INT4 expansion of the
+    // staged tile into the swizzled A layout; then signal the MMA (every tile,
+    // INT4 or not) and the epilogue.  Weights only: this role does not wait
+    // for the previous kernel.
+    const int xt = threadIdx.x - 32 * kFirstXfWarp;  // row of the 128-row block
+    const int sub = xt / a.bN;
+    const uint32_t g_total = cta_tiles(a);
+    RingPos sr{0, 0};
+    for (uint32_t g = 0; g < g_total; ++g) {
+      const int st = sr.i;
+      if (!__all_sync(0xffffffffu, mbar_wait(&staged[st], sr.ph, abort_flag))) {
+        fail(8);
+        break;
+      }
+      const uint32_t info = stage_info[st];
+      const uint32_t is4 = info & (info >> 2) & 3u;
+      const float swv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(stage_sc + st * 256)[xt]));
+      pre_sw[(g % kSwRing) * 128 + xt] = (info >> (2 + sub) & 1) ? swv * ((is4 >> sub & 1) ? 0.0625f : 1.0f) : 0.f;
+      for (int sb = 0; sb < a.tpb; ++sb) {
+        if (!(is4 >> sb & 1)) continue;
+        const uint8_t* src = stage_g(st) + sb * a.bN * (kTileK / 2);
+        uint8_t* dst = stage_a(st) + sb * a.bN * kTileK;
+        for (int q = xt; q < a.bN * 4; q += 32 * kXfWarps) {  // 16-byte source chunks
+          const int r8 = q >> 2, c4 = q & 3;
+          // 32 nibbles -> logical 16-byte chunks 2 c4 and 2 c4 + 1 of the 128-byte row
+          const uint4 v = *reinterpret_cast<const uint4*>(src + r8 * 64 + c4 * 16);
+          uint8_t* drow = dst + r8 * 128;
+          const uint2 e0 = expand8_x16(v.x), e1 = expand8_x16(v.y);
+          *reinterpret_cast<uint4*>(drow + (((2 * c4) ^ (r8 & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+          const uint2 e2 = expand8_x16(v.z), e3 = expand8_x16(v.w);
+          *reinterpret_cast<uint4*>(drow + (((2 * c4 + 1) ^ (r8 & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+        }
+      }
+      if (is4) fence_proxy_async_smem();  // generic-proxy writes -> visible to the MMA's async proxy
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&expanded[st]);
+        mbar_arrive(&sw_full[g % kSwRing]);
+      }
+      sr.next<S_>();
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     constexpr int kCols = Sh::kCols;
@@ -466,53 +511,8 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       if (lane == 0)
         for (int ab = 0; ab < kBufs; ++ab) mbar_arrive(&tmem_empty[ab]);
     }
-    // INT4 expansion: tiles ge .. last (this warp's share of each), then
-    // signal the MMA; every warp arrives for every tile, INT4 or not.  Each
-    // thread also stashes its row's weight scale of the tile (0 for a row past
-    // the layer's end; / 16 for INT4, whose codes were expanded as 16 q).
     const int et = threadIdx.x - 32 * kFirstEpiWarp;  // 0 .. 32 kEpiWarps - 1
-    uint32_t g_total = 0;                             // input tiles this CTA processes
-    for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
-      const Unit x = unit_of(a, u);
-      g_total += x.j1 - x.j0;
-    }
-    uint32_t ge = 0;
-    auto expand_upto = [&](uint32_t last) -> bool {
-      for (; ge <= last && ge < g_total; ++ge) {
-        const int st = ge % S_;
-        if (!__all_sync(0xffffffffu, mbar_wait(&staged[st], (ge / S_) & 1, abort_flag))) {
-          fail(8);
-          return false;
-        }
-        const uint32_t info = stage_info[st];
-        const uint32_t is4 = info & (info >> 2) & 3u;
-        {
-          const float swv = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(stage_sc + st * 256)[row]));
-          pre_sw[(ge % kSwRing) * 32 * Sh::kEpiWarps + et] =
-              (info >> (2 + sub) & 1) ? swv * ((is4 >> sub & 1) ? 0.0625f : 1.0f) : 0.f;
-        }
-        for (int sb = 0; sb < a.tpb; ++sb) {
-          if (!(is4 >> sb & 1)) continue;
-          const uint8_t* src = stage_g(st) + sb * a.bN * (kTileK / 2);
-          uint8_t* dst = stage_a(st) + sb * a.bN * kTileK;
-          for (int q = et; q < a.bN * 4; q += 32 * Sh::kEpiWarps) {  // 16-byte source chunks
-            const int r8 = q >> 2, c4 = q & 3;
-            // 32 nibbles -> logical 16-byte chunks 2 c4 and 2 c4 + 1 of the 128-byte row
-            const uint4 v = *reinterpret_cast<const uint4*>(src + r8 * 64 + c4 * 16);
-            uint8_t* drow = dst + r8 * 128;
-            const uint2 e0 = expand8_x16(v.x), e1 = expand8_x16(v.y);
-            *reinterpret_cast<uint4*>(drow + (((2 * c4) ^ (r8 & 7)) << 4)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-            const uint2 e2 = expand8_x16(v.z), e3 = expand8_x16(v.w);
-            *reinterpret_cast<uint4*>(drow + (((2 * c4 + 1) ^ (r8 & 7)) << 4)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
-          }
-        }
-        if (is4) fence_proxy_async_smem();  // generic-proxy writes -> visible to the MMA's async proxy
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&expanded[st]);
-      }
-      return true;
-    };
-    bool ok = expand_upto(kExpandAhead - 1);  // weights only: may overlap the previous kernel
+    bool ok = true;
     pdl_wait();  // outputs, token scales and workspace may still be in use by an earlier kernel
     const float2 nbias = make_float2(-kAccBiasF, -kAccBiasF);
     uint32_t g = 0, sync_phase = 0;
@@ -540,54 +540,57 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         // second tile's MMAs follows the first's, so one wait covers both
         const int nt = j + 1 < x.j1 ? 2 : 1;
         const uint32_t gl = g + nt - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[gl % kBufs], (gl / kBufs) & 1, abort_flag))) {
+        // the scale slot of the pair's last tile implies the first one's (the
+        // transform warps arrive in tile order)
+        if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[gl % kBufs], (gl / kBufs) & 1, abort_flag) &&
+                                         mbar_wait(&sw_full[gl % kSwRing], (gl / kSwRing) & 1, abort_flag))) {
           fail(9);
           ok = false;
           break;
         }
         tc_fence_after();
-        bool eok = true;
-        for (int k = 0; k < nt; ++k) {
-          const uint32_t gk = g + k;
-          const uint32_t taddr = tmem_base + ((uint32_t)(32 * quad) << 16) + (gk % kBufs) * NT + cg * kCols;
-          uint32_t v[Sh::kLdCols];
+        // the pair's accumulators in chunks of kLdCols columns, software
+        // pipelined: the load of chunk i + 1 is in flight while chunk i is
+        // rescaled (tcgen05.wait::ld waits for every load issued before it, so
+        // the next load is issued only after the wait for the current one)
+        constexpr int kL = Sh::kLdCols, kCpt = kCols / kL;
+        const uint32_t lane_base = tmem_base + ((uint32_t)(32 * quad) << 16) + cg * kCols;
+        const uint32_t taddr[2] = {lane_base + (g % kBufs) * NT, lane_base + ((g + 1) % kBufs) * NT};
+        float2 sw2[2];
 #pragma unroll
-          for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
-            tmem_ld16(taddr + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
-          // while the first loads are in flight: the INT4 expansion of later tiles
-          if (k == 0) eok = expand_upto(gl + kExpandAhead);
-          const float sw = pre_sw[(gk % kSwRing) * 32 * Sh::kEpiWarps + et];
-          const float2 sw2 = make_float2(sw, sw);
+        for (int k = 0; k < 2; ++k) {
+          const float sw = pre_sw[((g + k) % kSwRing) * 128 + row];  // slot g + 1 unused when nt == 1
+          sw2[k] = make_float2(sw, sw);
+        }
+        uint32_t v[2][kL];
+        tmem_ld16(taddr[0], v[0]);
+        const int nchunks = nt * kCpt;
 #pragma unroll
-          for (int c0 = 0; c0 < kCols; c0 += Sh::kLdCols) {
-            if (c0 > 0) {
-#pragma unroll
-              for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
-                tmem_ld16(taddr + c0 + c16 * 16, *reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
-            }
+        for (int i = 0; i < 2 * kCpt; ++i) {
+          if (i < nchunks) {
+            const int k = i / kCpt, c0 = (i % kCpt) * kL;
             tmem_wait_ld();
-#pragma unroll
-            for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16) tmem_regs_ready(*reinterpret_cast<uint32_t(*)[16]>(v + c16 * 16));
-#pragma unroll
-            for (int c16 = 0; c16 < Sh::kLdCols / 16; ++c16)
-              tmem_st16_const(taddr + c0 + c16 * 16, kAccBias);  // re-bias for the buffer's next use
+            tmem_regs_ready(v[i & 1]);
+            tmem_st16_const(taddr[k] + c0, kAccBias);  // re-bias for the buffer's next use
+            if (i + 1 < nchunks) tmem_ld16(taddr[(i + 1) / kCpt] + ((i + 1) % kCpt) * kL, v[(i + 1) & 1]);
             if constexpr (MODE == 2) {
               // INT4 label read back from the bitmap (debug path only)
               const int tt = (n / a.bN) * a.C + j + k;
               const bool t4 = rvalid && ((__ldg(a.bitmap + (tt >> 3)) >> (tt & 7)) & 1);
 #pragma unroll
-              for (int i = 0; i < Sh::kLdCols; ++i) {
-                const int m = mcol0 + c0 + i;
+              for (int e = 0; e < kL; ++e) {
+                const int m = mcol0 + c0 + e;
                 if (rvalid && m < a.M) {
-                  const int p16 = (int)(v[i] - kAccBias);
+                  const int p16 = (int)(v[i & 1][e] - kAccBias);
                   a.P[((size_t)m * a.N + n) * a.C + j + k] = t4 ? (p16 >> 4) : p16;
                 }
               }
             } else {
 #pragma unroll
-              for (int i = 0; i < Sh::kLdCols / 2; ++i) {
-                const float2 p = __fadd2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), nbias);
-                acc[c0 / 2 + i] = __ffma2_rn(p, sw2, acc[c0 / 2 + i]);
+              for (int e = 0; e < kL / 2; ++e) {
+                const float2 p =
+                    __fadd2_rn(make_float2(__uint_as_float(v[i & 1][2 * e]), __uint_as_float(v[i & 1][2 * e + 1])), nbias);
+                acc[c0 / 2 + e] = __ffma2_rn(p, sw2[k], acc[c0 / 2 + e]);
               }
             }
           }
@@ -601,10 +604,6 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         }
         g += nt;
         j += nt;
-        if (!eok) {
-          ok = false;
-          break;
-        }
       }
       if (!ok || MODE == 2) continue;
       cp_async_wait_all();
