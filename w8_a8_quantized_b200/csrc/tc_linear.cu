@@ -69,6 +69,7 @@ namespace {
 constexpr int kBufs = 4;        // accumulator buffers in tensor memory
 constexpr int kSwRing = 16;     // ring of per-row weight scales, one slot per tile (> stages + kBufs)
 constexpr int kMetaSlots = 32;  // metadata ring slots (one per lane of the metadata warp)
+constexpr int kDone = 16;       // MMA-completion barriers, one per tile, reused every kDone tiles
 constexpr int kFirstXfWarp = 4;   // transform warps: INT4 expansion and per-row weight scales
 constexpr int kXfWarps = 4;       // 128 threads, one per row of the 128-row block
 constexpr int kFirstEpiWarp = kFirstXfWarp + kXfWarps;
@@ -108,6 +109,9 @@ struct TcShape {
   // (a stage is refilled only after its MMAs, which wait for an accumulator
   // buffer the epilogue released), so a scale slot is never rewritten early
   static_assert(kStages + kBufs < kSwRing, "scale ring depth");
+  // a tile's completion barrier is waited for (by the epilogue, and by the
+  // producers refilling its stage) before the MMA can complete tile + kDone
+  static_assert(kDone > kStages && kDone > kBufs, "completion ring depth");
   static_assert(kThreads <= 1024, "block size");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -266,9 +270,10 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
   uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);  // weights (INT8) + activations landed; one arrival per producer
   uint64_t* staged = full + S_;                        // INT4 staging landed (0 bytes when none)
   uint64_t* expanded = staged + S_;                    // transform warps done with the stage (one arrival each)
-  uint64_t* empty = expanded + S_;                     // MMAs reading the stage done
-  uint64_t* tmem_full = empty + S_;
-  uint64_t* tmem_empty = tmem_full + kBufs;
+  // mma_done[g % kDone]: the MMAs of tile g are complete (one commit per tile):
+  // its stage may be refilled and its accumulator buffer read
+  uint64_t* mma_done = expanded + S_;
+  uint64_t* tmem_empty = mma_done + kDone;
   uint64_t* meta_full = tmem_empty + kBufs;
   uint64_t* meta_empty = meta_full + kMetaSlots;
   uint64_t* epi_sync = meta_empty + kMetaSlots;  // epilogue-only rendezvous (bounded, unlike bar.sync)
@@ -283,7 +288,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
   float* pre_bias = reinterpret_cast<float*>(ctrl + Sh::kCtrlBytes);  // [32 kEpiWarps] bias of each epilogue row
   float* pre_sx = pre_bias + 32 * Sh::kEpiWarps;                       // [kEpiWarps][kCols] token scales
   float* pre_sw = pre_sx + Sh::kEpiWarps * Sh::kCols;                    // [kSwRing][128] weight scale of each row
-  static_assert((4 * 8 + 2 * kBufs + 2 * kMetaSlots + 2 + kSwRing) * 8 + kMetaSlots * 16 + (8 + 4) * 4 <=
+  static_assert((3 * 8 + kDone + kBufs + 2 * kMetaSlots + 2 + kSwRing) * 8 + kMetaSlots * 16 + (8 + 4) * 4 <=
                     Sh::kCtrlBytes,
                 "control area");
 
@@ -293,12 +298,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       mbar_init(&full[st], 2);
       mbar_init(&staged[st], 1);
       mbar_init(&expanded[st], kXfWarps);
-      mbar_init(&empty[st], 1);
     }
     for (int b = 0; b < kBufs; ++b) {
-      mbar_init(&tmem_full[b], 1);
       mbar_init(&tmem_empty[b], Sh::kEpiWarps);
     }
+    for (int i = 0; i < kDone; ++i) mbar_init(&mma_done[i], 1);
     for (int s = 0; s < kMetaSlots; ++s) {
       mbar_init(&meta_full[s], 1);
       mbar_init(&meta_empty[s], 1);
@@ -339,7 +343,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         const MetaRec rec = meta[mr.i];
         mbar_arrive(&meta_empty[mr.i]);
         mr.next<kMetaSlots>();
-        if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(2); ok = false; break; }
+        if (g >= (uint32_t)S_ && !mbar_wait(&mma_done[(g - S_) % kDone], ((g - S_) / kDone) & 1, abort_flag)) {
+          fail(2);
+          ok = false;
+          break;
+        }
         const uint32_t kinds = rec.sizes >> 28;
         const uint32_t sc_bytes = (kinds & 8) ? 4u * a.bN : 2u * a.bN;  // fp16 row scales of the tile's sub-tiles
         stage_info[sr.i] = kinds;  // read by the transform warps after `staged`
@@ -378,8 +386,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
 #pragma unroll
         for (int k = 0; k < kTileK / 32; ++k)  // K = 32 bytes per instruction: +2 in 16-byte units
           mma_i8(d, adesc0 + soff + 2 * k, bdesc0 + soff + 2 * k, Sh::kIdesc, 1u);
-        mma_commit(&empty[sr.i]);
-        mma_commit(&tmem_full[br.i]);
+        mma_commit(&mma_done[g % kDone]);
         sr.next<S_>();
         br.next<kBufs>();
       }
@@ -436,7 +443,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       RingPos sr{0, 0};
       bool ok = true;
       for (uint32_t g = 0; g < g_total; ++g, bi.next(a)) {
-        if (!mbar_wait(&empty[sr.i], sr.ph ^ 1, abort_flag)) { fail(3); ok = false; break; }
+        if (g >= (uint32_t)S_ && !mbar_wait(&mma_done[(g - S_) % kDone], ((g - S_) / kDone) & 1, abort_flag)) {
+          fail(3);
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&full[sr.i], Sh::kB);
         tma_load_2d(stage_b(sr.i), &tm_x, bi.j * kTileK, bi.x.tb * NT, &full[sr.i]);
         sr.next<S_>();
@@ -542,7 +553,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         const uint32_t gl = g + nt - 1;
         // the scale slot of the pair's last tile implies the first one's (the
         // transform warps arrive in tile order)
-        if (!__all_sync(0xffffffffu, mbar_wait(&tmem_full[gl % kBufs], (gl / kBufs) & 1, abort_flag) &&
+        if (!__all_sync(0xffffffffu, mbar_wait(&mma_done[gl % kDone], (gl / kDone) & 1, abort_flag) &&
                                          mbar_wait(&sw_full[gl % kSwRing], (gl / kSwRing) & 1, abort_flag))) {
           fail(9);
           ok = false;
