@@ -183,6 +183,34 @@ int aq_quantize_weights(const void* w, int wdtype, int N, int K, int ldw, int bN
 int aq_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream);
 
 /*
+ * Long-prefill variant (App. E.2, E.3): the paper expands a mixed projection
+ * once per call into a temporary INT8 buffer and then runs a pure INT8 GEMM.
+ *
+ * aq_expanded_bytes: host only; bytes of the all-INT8 copy of *w (payload
+ * R*C*bN*bK, tile table 4*R*C, two offset arrays 4*(R+1) each, bitmap
+ * ceil(R*C/8), each rounded up to 256 bytes); 0 when *w is invalid.
+ *
+ * aq_expand_int8: writes that copy into the caller's device buffer `buf`
+ * (256-byte aligned, >= aq_expanded_bytes bytes) and describes it in *out
+ * (host struct): T4 = 0, every tile INT8 (INT4 codes sign-extended, INT8
+ * tiles copied), tile (r, j) at index r*C + j, and out->scales = w->scales
+ * (shared, not copied).  *out is valid while `buf` and w's scales live.
+ * Asynchronous on `stream`; no allocation, no synchronization.
+ * Errors: AQ_ERR_ARG (null or misaligned pointer), AQ_ERR_SHAPE,
+ * AQ_ERR_WORKSPACE (buffer too small), AQ_ERR_CUDA.
+ *
+ * aq_linear_prefill_expanded: aq_linear_prefill with the expansion done
+ * first into `tmp` (as aq_expand_int8, tmp_bytes >= aq_expanded_bytes(w)),
+ * both kernels on `stream`.  The results equal aq_linear_prefill's bit for
+ * bit.  Errors: as aq_linear_prefill, plus AQ_ERR_ARG / AQ_ERR_WORKSPACE for tmp.
+ */
+size_t aq_expanded_bytes(const aq_packed* w);
+int aq_expand_int8(const aq_packed* w, void* buf, size_t buf_bytes, aq_packed* out, void* stream);
+int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                               void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* tmp, size_t tmp_bytes,
+                               void* stream);
+
+/*
  * Device scratch bytes a linear call needs for `phase` (aq_phase) at M tokens
  * with packed weights *w (host struct; only its geometry is read).  Host only.
  * The workspace must be zero-filled once when allocated; afterwards the library

@@ -198,3 +198,24 @@ def test_paper_accounting_matches_oracle_and_rejects(R, C, T4, bN, bK):
     assert L.aq_paper_packed_bytes(R, C, T4, 3, 3, ctypes.byref(out)) == -1
     assert L.aq_paper_packed_bytes(0, C, 0, bN, bK, ctypes.byref(out)) == -1
     assert L.aq_paper_packed_bytes(R, C, T4, bN, bK, None) == -1
+
+
+def test_long_prefill_sizes_and_validation():
+    L = aq.lib()
+    s = aq.AqPackedStruct(N=256, K=384, bN=128, bK=128, R=2, C=3, T4=2, T8=4,
+                          bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    a256 = lambda b: (b + 255) // 256 * 256
+    want = a256(6 * 128 * 128) + a256(4 * 6) + 2 * a256(4 * 3) + a256(1)
+    assert L.aq_expanded_bytes(ctypes.byref(s)) == want
+    bad = aq.AqPackedStruct(N=100, K=384, bN=128, bK=128, R=0, C=3, T4=0, T8=0)
+    assert L.aq_expanded_bytes(ctypes.byref(bad)) == 0
+    out = aq.AqPackedStruct()
+    assert L.aq_expand_int8(ctypes.byref(s), None, want, ctypes.byref(out), None) == -1
+    assert L.aq_expand_int8(ctypes.byref(s), 4096 + 16, want, ctypes.byref(out), None) == -1  # not 256-byte aligned
+    assert L.aq_expand_int8(ctypes.byref(s), 4096, want - 1, ctypes.byref(out), None) == -5
+    assert L.aq_expand_int8(ctypes.byref(bad), 4096, want, ctypes.byref(out), None) == -2
+    ws = L.aq_workspace_bytes(1, 300, ctypes.byref(s))
+    f = L.aq_linear_prefill_expanded
+    assert f(ctypes.byref(s), 16, 16, 300, None, 16, 0, 256, 16, ws, None, want, None) == -1
+    assert f(ctypes.byref(s), 16, 16, 300, None, 16, 0, 256, 16, ws, 4096, want - 1, None) == -5
+    assert f(ctypes.byref(s), 16, 16, 300, None, 16, 0, 256, 16, ws - 1, 4096, want, None) == -5

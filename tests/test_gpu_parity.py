@@ -397,3 +397,34 @@ def test_quantize_and_pack_feeds_the_linear_layer(M):
     y = (aq.aq_linear_decode if M <= 64 else aq.aq_linear_prefill)(pw, xq, sx)
     ref_p = synth.SingleProjection(N, K, bN, 128, pmap, rc, rs)
     assert_output_close(y, oracle_linear(ref_p, x))
+
+
+# ------------------------------------------------------------------ long-prefill variant
+
+@pytest.mark.parametrize("N,K,bN,frac8", [(256, 384, 128, 0.5), (192, 512, 64, 0.3), (128, 256, 128, 0.0),
+                                          (384, 256, 64, 1.0)])
+def test_expand_int8_matches_oracle_codes(N, K, bN, frac8):
+    p = synth.projection_inputs(N, K, bN, 128, frac8, (71, N))
+    w = aq.aq_pack(*dev_projection(p), bN, 128)
+    e = aq.ExpandedWeights(w)
+    torch.cuda.synchronize()
+    R, C = N // bN, K // 128
+    assert (e.T4, e.T8) == (0, R * C)
+    got = e.host_buffers()
+    codes, _, _ = oracle.unpack(oracle.pack(p.codes, p.scales, p.pmap, bN, 128))
+    want = codes.reshape(R, bN, C, 128).transpose(0, 2, 1, 3).reshape(R * C, bN, 128).astype(np.int8)
+    assert np.array_equal(got["w8"], want)
+    assert not got["bitmap"].any() and not got["row_off4"].any()
+    assert np.array_equal(got["row_off8"], np.arange(R + 1) * C)
+    assert np.array_equal(got["tile_idx"], np.arange(R * C))
+
+
+@pytest.mark.parametrize("M,bN,frac8,out_dtype", [(300, 128, 0.4, torch.float32), (1, 64, 0.3, torch.float32),
+                                                  (700, 64, 0.25, torch.bfloat16), (129, 128, 0.0, torch.float32)])
+def test_prefill_expanded_equals_prefill_bit_for_bit(M, bN, frac8, out_dtype):
+    p, x, w, xq, sx = packed_case(512, 768, bN, frac8, 73, M, outlier=0.01)
+    bias = torch.from_numpy(np.random.default_rng(74).standard_normal(512).astype(np.float32)).cuda()
+    y1 = aq.aq_linear_prefill(w, xq, sx, bias=bias, out_dtype=out_dtype)
+    y2 = aq.aq_linear_prefill_expanded(w, xq, sx, bias=bias, out_dtype=out_dtype)
+    assert torch.equal(y1, y2)
+    assert_output_close(y2, oracle_linear(p, x, bias=bias.cpu().numpy()))

@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -22,7 +23,8 @@ BUF_NAMES = ("bitmap", "row_off4", "row_off8", "tile_idx", "w4", "w8", "scales")
 EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "aq_quant_act",
             "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
             "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc",
-            "aq_quantize_weights", "aq_paper_packed_bytes")
+            "aq_quantize_weights", "aq_paper_packed_bytes", "aq_expanded_bytes", "aq_expand_int8",
+            "aq_linear_prefill_expanded")
 
 
 class AqError(RuntimeError):
@@ -62,6 +64,13 @@ def lib():
     L.aq_quant_act.restype = c_int
     L.aq_paper_packed_bytes.restype = c_int
     L.aq_paper_packed_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_size_t)]
+    L.aq_expanded_bytes.restype = c_size_t
+    L.aq_expanded_bytes.argtypes = [P]
+    L.aq_expand_int8.restype = c_int
+    L.aq_expand_int8.argtypes = [P, c_void_p, c_size_t, P, c_void_p]
+    L.aq_linear_prefill_expanded.restype = c_int
+    L.aq_linear_prefill_expanded.argtypes = [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p,
+                                             c_size_t, c_void_p, c_size_t, c_void_p]
     L.aq_quantize_weights.restype = c_int
     L.aq_quantize_weights.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_int,
                                       c_void_p, c_void_p, c_void_p]
@@ -261,6 +270,63 @@ def aq_linear_prefill(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=t
     """Prefill-phase y (tensor-core INT8 path), any M >= 1."""
     return _linear(lib().aq_linear_prefill, "aq_linear_prefill", AQ_PHASE_PREFILL, w, xq, sx, bias, out, out_dtype,
                    ws)
+
+
+def aq_expanded_bytes(w: PackedWeights) -> int:
+    """Bytes of the all-INT8 copy of w made by the long-prefill variant."""
+    return int(lib().aq_expanded_bytes(ctypes.byref(w.struct)))
+
+
+class ExpandedWeights:
+    """The all-INT8 copy of a packed projection (long-prefill variant); shares w's scales."""
+
+    def __init__(self, w: PackedWeights, buf: torch.Tensor = None):
+        need = aq_expanded_bytes(w)
+        if need == 0:
+            raise ValueError("invalid packed weights")
+        self.source, self.device = w, w.device
+        self.buf = torch.empty(need + 256, dtype=torch.uint8, device=w.device) if buf is None else buf
+        off = (-self.buf.data_ptr()) % 256  # the library wants a 256-byte aligned buffer
+        self.base = self.buf[off:off + need]
+        self.struct = AqPackedStruct()
+        _check(lib().aq_expand_int8(ctypes.byref(w.struct), self.base.data_ptr(), need, ctypes.byref(self.struct),
+                                    _stream(w.device)), "aq_expand_int8")
+
+    N = property(lambda s: s.struct.N)
+    K = property(lambda s: s.struct.K)
+    R = property(lambda s: s.struct.R)
+    C = property(lambda s: s.struct.C)
+    T4 = property(lambda s: s.struct.T4)
+    T8 = property(lambda s: s.struct.T8)
+
+    def host_buffers(self) -> dict:
+        """Bitmap, offsets, tile table and INT8 payload as host arrays (scales: the source's)."""
+        st, R, C, bN = self.struct, self.R, self.C, self.struct.bN
+        T = R * C
+        def view(ptr, nbytes):
+            o = ptr - self.base.data_ptr()
+            return self.base[o:o + nbytes].cpu().numpy()
+        return {"bitmap": view(st.bitmap, (T + 7) // 8), "row_off4": view(st.row_off4, 4 * (R + 1)).view(np.int32),
+                "row_off8": view(st.row_off8, 4 * (R + 1)).view(np.int32),
+                "tile_idx": view(st.tile_idx, 4 * T).view(np.int32),
+                "w8": view(st.w8, T * bN * 128).view(np.int8).reshape(T, bN, 128)}
+
+
+def aq_linear_prefill_expanded(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=torch.float32, ws=None,
+                               tmp=None):
+    """aq_linear_prefill through the long-prefill variant: expand to an INT8 copy in
+    `tmp` (uint8, >= aq_expanded_bytes(w) + 256), then the pure INT8 GEMM."""
+    need = aq_expanded_bytes(w)
+    if tmp is None:
+        tmp = torch.empty(need + 256, dtype=torch.uint8, device=w.device)
+    off = (-tmp.data_ptr()) % 256
+    if tmp.numel() - off < need:
+        raise ValueError("tmp is too small")
+    L = lib()
+    def fn(wp, xqp, sxp, M, bp, yp, ydt, ldy, wsp, wsn, st):
+        return L.aq_linear_prefill_expanded(wp, xqp, sxp, M, bp, yp, ydt, ldy, wsp, wsn, tmp.data_ptr() + off,
+                                            tmp.numel() - off, st)
+    return _linear(fn, "aq_linear_prefill_expanded", AQ_PHASE_PREFILL, w, xq, sx, bias, out, out_dtype, ws)
 
 
 def aq_linear_decode_noalloc(w: PackedWeights, xq, sx, bias=None, out=None, out_dtype=torch.float32):

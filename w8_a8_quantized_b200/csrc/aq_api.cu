@@ -153,6 +153,33 @@ extern "C" int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const flo
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
 }
 
+extern "C" size_t aq_expanded_bytes(const aq_packed* w) {
+  return validate_packed(w) == AQ_OK ? expanded_bytes(w) : 0;
+}
+
+extern "C" int aq_expand_int8(const aq_packed* w, void* buf, size_t buf_bytes, aq_packed* out, void* stream) {
+  int rc = validate_packed(w);
+  if (rc != AQ_OK) return rc;
+  if (!buf || !out || ((uintptr_t)buf & 255)) return AQ_ERR_ARG;
+  if (buf_bytes < expanded_bytes(w)) return AQ_ERR_WORKSPACE;
+  return launch_expand_int8(w, buf, out, static_cast<cudaStream_t>(stream)) == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+}
+
+extern "C" int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, const float* sx, int M,
+                                          const float* bias, void* y, int ydtype, int ldy, void* ws, size_t ws_bytes,
+                                          void* tmp, size_t tmp_bytes, void* stream) {
+  int rc = check_linear(w, xq, sx, M, y, ydtype, ldy);
+  if (rc != AQ_OK) return rc;
+  if (!ws || ws_bytes < prefill_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
+  if (!tmp || ((uintptr_t)tmp & 255)) return AQ_ERR_ARG;
+  if (tmp_bytes < expanded_bytes(w)) return AQ_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  aq_packed e;
+  cudaError_t err = launch_expand_int8(w, tmp, &e, st);
+  if (err == cudaSuccess) err = launch_tc(&e, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_PREFILL, st);
+  return err == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+}
+
 extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int M, int phase, int32_t* P, void* ws,
                                       size_t ws_bytes, void* stream) {
   int rc = validate_packed(w);

@@ -75,6 +75,9 @@ size_t prefill_ws_bytes(int M, const aq_packed* w);
 cudaError_t launch_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, cudaStream_t st);
 cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, const aq_packed* out,
                                 const uint8_t* map_dev, int* err_dev, cudaStream_t st);
+// Long-prefill variant: all-INT8 copy of a packed projection in a caller buffer.
+size_t expanded_bytes(const aq_packed* w);
+cudaError_t launch_expand_int8(const aq_packed* w, void* buf, aq_packed* out, cudaStream_t st);
 cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
                       int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st);
 
