@@ -55,7 +55,7 @@ size_t decode_ws_bytes(int M, const aq_packed* w) {
   const DecodePlan p = plan_decode(M, w);
   if (p.kernel == 0) return kWsHeader;
   size_t b = kWsHeader + counters_bytes(p.blocks);
-  if (p.S > 1) b += (size_t)p.S * M * w->N * sizeof(float);
+  if (p.S > 1) b += (size_t)p.S * ((M + 3) & ~3) * w->N * sizeof(float);  // [S][N][M rounded up to 4]
   return b;
 }
 

@@ -70,6 +70,7 @@ constexpr int kBufs = 4;        // accumulator buffers in tensor memory
 constexpr int kSwRing = 16;     // ring of per-row weight scales, one slot per tile (> stages + kBufs)
 constexpr int kMetaSlots = 32;  // metadata ring slots (one per lane of the metadata warp)
 constexpr int kDone = 16;       // MMA-completion barriers, one per tile, reused every kDone tiles
+constexpr int kMaxTcSplits = 8;  // split-K bound of the decode plan (the reduction unrolls over it)
 constexpr int kFirstXfWarp = 4;   // transform warps: INT4 expansion and per-row weight scales
 constexpr int kXfWarps = 4;       // 128 threads, one per row of the 128-row block
 constexpr int kFirstEpiWarp = kFirstXfWarp + kXfWarps;
@@ -134,7 +135,7 @@ struct TcArgs {
   void* y;
   int ydtype, ldy;
   void* ws;
-  float* partial;  // [S][M][N]
+  float* partial;  // [S][N][Mp], Mp = M rounded up to a multiple of 4
   int* counters;   // [nrb * ntb]
   int32_t* P;      // debug: exact tile products [M][N][C], or null
 };
@@ -249,6 +250,51 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void abort_grace() {
   const unsigned long long t0 = globaltimer_ns();
   while (globaltimer_ns() - t0 < kAbortGraceNs) __nanosleep(1000);
+}
+
+// Largest multiple of 4 that divides kCols and is at most lim.
+constexpr int chunk_cols(int kCols, int lim) {
+  int c = lim;
+  while (c > 4 && kCols % c != 0) c -= 4;
+  return c;
+}
+
+// Sum of the S split partials of a thread's kCols columns (split order
+// increasing), scaled by the token scales, plus bias, stored.  CH columns at a
+// time with the loads of all (at most SMAX) splits in flight together.
+template <int kCols, int CH, int SMAX>
+__device__ __forceinline__ void reduce_splits(const TcArgs& a, const float* prow, size_t sstride, int mcol0, int n,
+                                              float bias_n) {
+  static_assert(kCols % CH == 0 && CH % 4 == 0, "reduction chunks");
+#pragma unroll 1
+  for (int c0 = 0; c0 < kCols; c0 += CH) {
+    float4 v[SMAX][CH / 4];
+#pragma unroll
+    for (int ss = 0; ss < SMAX; ++ss)
+#pragma unroll
+      for (int i4 = 0; i4 < CH / 4; ++i4)
+        v[ss][i4] = (ss < a.S && mcol0 + c0 + 4 * i4 < a.M)
+                        ? __ldcg(reinterpret_cast<const float4*>(prow + ss * sstride + c0) + i4)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i4 = 0; i4 < CH / 4; ++i4) {
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int ss = 0; ss < SMAX; ++ss)
+        if (ss < a.S) {
+          sum.x += v[ss][i4].x;
+          sum.y += v[ss][i4].y;
+          sum.z += v[ss][i4].z;
+          sum.w += v[ss][i4].w;
+        }
+      const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = mcol0 + c0 + 4 * i4 + e;
+        if (m < a.M) store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sv[e], bias_n));
+      }
+    }
+  }
 }
 
 // MODE: 0 = outputs written directly (one split), 1 = split-K partial sums
@@ -652,14 +698,18 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         __syncwarp();  // the scale slots are rewritten at the next unit's start
         continue;
       }
-      // split-K: publish the partial sum, the last CTA of this unit group reduces
+      // split-K: publish the partial sum, the last CTA of this unit group reduces.
+      // Partials are [S][N][Mp] (Mp = M rounded up to 4): a thread's columns
+      // are contiguous, written and read as 16-byte vectors.
+      const int Mp = (a.M + 3) & ~3;
+      float* const prow = a.partial + (size_t)n * Mp + mcol0;  // this thread's split-0 columns
+      const size_t sstride = (size_t)a.N * Mp;
       if (rvalid) {
 #pragma unroll
-        for (int i = 0; i < kCols; ++i) {
-          const int m = mcol0 + i;
-          const float s = i & 1 ? acc[i / 2].y : acc[i / 2].x;
-          if (m < a.M) __stcg(a.partial + ((size_t)x.s * a.M + m) * a.N + n, s);
-        }
+        for (int i4 = 0; i4 < kCols / 4; ++i4)
+          if (mcol0 + 4 * i4 < a.M)
+            __stcg(reinterpret_cast<float4*>(prow + x.s * sstride) + i4,
+                   make_float4(acc[2 * i4].x, acc[2 * i4].y, acc[2 * i4 + 1].x, acc[2 * i4 + 1].y));
       }
       __threadfence();
       mbar_arrive(epi_sync);
@@ -672,22 +722,12 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       if (*last_flag) {
         __threadfence();
         if (rvalid) {
-          // splits outer, columns inner: the kCols loads of a split are independent
-          // and all in flight together (split order stays increasing)
-          float sum[kCols];
-#pragma unroll
-          for (int i = 0; i < kCols; ++i) sum[i] = 0.f;
-          for (int ss = 0; ss < a.S; ++ss) {
-            const float* ps = a.partial + (size_t)ss * a.M * a.N + n;
-#pragma unroll
-            for (int i = 0; i < kCols; ++i)
-              if (mcol0 + i < a.M) sum[i] += __ldcg(ps + (size_t)(mcol0 + i) * a.N);
-          }
-#pragma unroll
-          for (int i = 0; i < kCols; ++i) {
-            const int m = mcol0 + i;
-            if (m < a.M) store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sum[i], bias_n));
-          }
+          // the loads of every split for a chunk of columns are issued before any
+          // of them is summed, then the splits are added in increasing order;
+          // chunks are as wide as 64 values in flight allow
+          if (a.S <= 2) reduce_splits<kCols, chunk_cols(kCols, 32), 2>(a, prow, sstride, mcol0, n, bias_n);
+          else if (a.S <= 4) reduce_splits<kCols, chunk_cols(kCols, 16), 4>(a, prow, sstride, mcol0, n, bias_n);
+          else reduce_splits<kCols, chunk_cols(kCols, 8), kMaxTcSplits>(a, prow, sstride, mcol0, n, bias_n);
         }
         if (ew == 0 && lane == 0) a.counters[x.rb * a.ntb + x.tb] = 0;
       }
@@ -778,6 +818,7 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
   if (phase == AQ_PHASE_DECODE && P == nullptr) {
     const DecodePlan p = plan_decode(M, w);
     a.S = p.S;
+    if (a.S > kMaxTcSplits) return cudaErrorInvalidValue;  // the split reduction unrolls over kMaxTcSplits
     const size_t cnt_bytes = ((size_t)p.blocks * sizeof(int) + 255) / 256 * 256;
     a.partial = reinterpret_cast<float*>(wsb + kWsHeader + cnt_bytes);
   } else {
