@@ -239,8 +239,10 @@ class Model:
         if self.phase == aq.AQ_PHASE_PREFILL:
             need = max(aq.aq_expanded_bytes(w) for layer in self.weights for w in layer.values())
             self.tmp = torch.empty(need + 256, dtype=torch.uint8, device=self.dev)
-        # input kinds whose group runs as one fused launch (activation preparation inside)
-        self.fused = self.phase == aq.AQ_PHASE_DECODE and M <= 8
+        # groups run as one fused launch (activation preparation inside) up to 2 tokens; from
+        # 3 tokens on as one preparation launch plus one grouped CUDA-core launch (up to 4 tokens,
+        # or up to 8 for groups of three or more) or one tensor-core launch per member
+        self.fused = self.phase == aq.AQ_PHASE_DECODE and M <= 2
 
     def step(self, mode="group"):
         """Enqueue one pass; returns the number of kernel launches.
@@ -256,7 +258,8 @@ class Model:
             for kind, names in self.members.items():
                 if mode == "group":
                     self.groups[l][kind](self.x[l][kind], [self.y[nm] for nm in names], ws=self.ws)
-                    n += 1 if self.fused else 1 + len(names)  # fused launch, or quantize + members
+                    rows = self.phase == aq.AQ_PHASE_DECODE and (self.M <= 4 or (len(names) >= 3 and self.M <= 8))
+                    n += 1 if self.fused else 1 + (1 if rows else len(names))  # fused, or quantize + members
                 elif mode == "expanded":
                     for nm in names:
                         aq.aq_linear_prefill_expanded(self.weights[l][nm], self.xq[kind], self.sx[kind],

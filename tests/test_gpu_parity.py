@@ -220,8 +220,9 @@ def test_decode_wide_layer_matches_oracle(M):
 
 
 @pytest.mark.parametrize("M", [1, 2, 5, 8, 9, 24, 64])
-def test_group_decode_matches_separate_calls_and_oracle(M):
-    shapes = [(768, 1024), (256, 1024), (256, 1024)]
+@pytest.mark.parametrize("members", [3, 2])
+def test_group_decode_matches_separate_calls_and_oracle(M, members):
+    shapes = [(768, 1024), (256, 1024), (256, 1024)][:members]
     ps, ws, x = _group_case(shapes, M, 1000 + M, aq.AQ_PHASE_DECODE)
     xd = dev_bf16(x)
     grp = aq.Group(ws, aq.AQ_PHASE_DECODE, M)
@@ -231,8 +232,13 @@ def test_group_decode_matches_separate_calls_and_oracle(M):
     xq, sx = aq.aq_quant_act(xd)
     for g, (p, w) in enumerate(zip(ps, ws)):
         sep = aq.aq_linear_decode(w, xq, sx, bias=biases[g])
-        assert torch.equal(outs[g], sep), g
+        # a group of three or more runs as one CUDA-core launch up to 8 tokens, where a
+        # single call from 5 tokens on takes the tensor cores: same products, different
+        # FP32 summation order, so only the oracle comparison applies there
+        if not (members >= 3 and 5 <= M <= 8):
+            assert torch.equal(outs[g], sep), g
         assert_output_close(outs[g], oracle_linear(p, x, bias=biases[g].cpu().numpy()))
+        assert_output_close(sep, oracle_linear(p, x, bias=biases[g].cpu().numpy()))
     aq.check_all_workspaces()
     rc, _ = aq.aq_workspace_status(grp.ws)
     assert rc == 0

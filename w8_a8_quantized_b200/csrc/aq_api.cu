@@ -28,12 +28,16 @@ static constexpr int kMaxSplits = 8;
 // preparation grows with M).  The fused codes live in shared memory.
 bool rows_fusable(int M, int K) { return M <= 2 && 2 * (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
 
-// Decode: up to 8 tokens on the CUDA cores (bandwidth-bound, one CTA per 32
+// Decode: up to 4 tokens on the CUDA cores (bandwidth-bound, one CTA per 32
 // output rows, no split); more tokens on the tensor cores with splits over
-// tile columns to fill the GPU in one wave.
+// tile columns to fill the GPU in one wave.  (Groups of three or more
+// projections keep one grouped CUDA-core launch up to kRowsMaxM tokens: see
+// group_rows.)
+static constexpr int kRowsPreferM = 4;
+
 DecodePlan plan_decode(int M, const aq_packed* w) {
   DecodePlan p;
-  if (rows_supported(M, w->K)) {
+  if (rows_supported(M, w->K) && M <= kRowsPreferM) {
     p.kernel = 0;
     p.rows = 16;
     p.blocks = w->N / 16;
@@ -229,6 +233,20 @@ static size_t group_ws_bytes(int phase, int M, const aq_packed* const* w, int G)
   return align256(lin) + align256((size_t)M * w[0]->K) + align256((size_t)M * sizeof(float));
 }
 
+// A decode group runs as one CUDA-core launch over all members' rows when every
+// member would use the CUDA-core kernel alone, or, up to kRowsMaxM tokens,
+// when it has three or more members (one launch beats one tensor-core launch
+// per member there: q/k/v at 8 tokens, 24.8 against 27.6 us per layer).
+static bool group_rows(int phase, const aq_packed* const* w, int G, int M) {
+  if (phase != AQ_PHASE_DECODE) return false;
+  bool all_rows = true, all_supported = true;
+  for (int g = 0; g < G; ++g) {
+    all_rows = all_rows && plan_decode(M, w[g]).kernel == 0;
+    all_supported = all_supported && rows_supported(M, w[g]->K);
+  }
+  return all_rows || (G >= 3 && all_supported);
+}
+
 extern "C" size_t aq_group_workspace_bytes(int phase, int M, const aq_packed* const* w, int G) {
   if (!w || G < 1 || G > kMaxGroup || M < 1) return 0;
   if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return 0;
@@ -265,9 +283,7 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   int8_t* xq = reinterpret_cast<int8_t*>(base + align256(lin));
   float* sx = reinterpret_cast<float*>(base + align256(lin) + align256((size_t)M * K));
   e = launch_quant_act(x, M, K, ldx, xq, sx, st);
-  bool rows_all = phase == AQ_PHASE_DECODE;
-  for (int g = 0; g < G; ++g) rows_all = rows_all && plan_decode(M, w[g]).kernel == 0;
-  if (e == cudaSuccess && rows_all) {  // one CUDA-core launch over all members' rows
+  if (e == cudaSuccess && group_rows(phase, w, G, M)) {  // one CUDA-core launch over all members' rows
     DecodeProj d[kMaxGroup];
     for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
     e = launch_decode_rows(d, G, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
