@@ -266,6 +266,7 @@ template <int kCols, int CH, int SMAX>
 __device__ __forceinline__ void reduce_splits(const TcArgs& a, const float* prow, size_t sstride, int mcol0, int n,
                                               float bias_n) {
   static_assert(kCols % CH == 0 && CH % 4 == 0, "reduction chunks");
+  const bool sx_vec = ((uintptr_t)a.sx & 15) == 0;
 #pragma unroll 1
   for (int c0 = 0; c0 < kCols; c0 += CH) {
     float4 v[SMAX][CH / 4];
@@ -288,11 +289,18 @@ __device__ __forceinline__ void reduce_splits(const TcArgs& a, const float* prow
           sum.w += v[ss][i4].w;
         }
       const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+      const int m0 = mcol0 + c0 + 4 * i4;
+      float xs[4];
+      if (sx_vec && m0 + 3 < a.M) {  // four token scales in one load
+        const float4 q = __ldg(reinterpret_cast<const float4*>(a.sx + m0));
+        xs[0] = q.x; xs[1] = q.y; xs[2] = q.z; xs[3] = q.w;
+      } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int m = mcol0 + c0 + 4 * i4 + e;
-        if (m < a.M) store_y(a.y, a.ydtype, (size_t)m * a.ldy + n, fmaf(__ldg(a.sx + m), sv[e], bias_n));
+        for (int e = 0; e < 4; ++e) xs[e] = m0 + e < a.M ? __ldg(a.sx + m0 + e) : 0.f;
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (m0 + e < a.M) store_y(a.y, a.ydtype, (size_t)(m0 + e) * a.ldy + n, fmaf(xs[e], sv[e], bias_n));
     }
   }
 }
