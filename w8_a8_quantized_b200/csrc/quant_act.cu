@@ -4,17 +4,21 @@
 // for the CUDA preparation step (see quant_code for the exact fast path).
 //
 // One CTA per token row.  Each thread owns 16-byte vectors (8 bf16) of the row:
-// pass 1 reduces max|x| (kept in registers for rows up to 32768 features),
+// pass 1 reduces max|x| (kept in registers for rows up to CV x 2048 features),
 // pass 2 writes the codes as 8-byte stores.  HBM traffic: 2 bytes read and 1
-// byte written per element, plus 4 bytes per row.
+// byte written per element, plus 4 bytes per row.  The register cache is sized
+// to the row (CV = 1..16 vectors per thread): a fixed 16-vector cache held a
+// 2560-feature row's CTA to two per SM, and the latency-bound per-row chain
+// then ran at a fraction of HBM bandwidth.
 #include "aq_internal.cuh"
 
 namespace aq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kCachedVecs = 16;  // 16 x 256 x 8 = 32768 features held in registers
+constexpr int kMaxCachedVecs = 16;  // 16 x 256 x 8 = 32768 features held in registers
 
+template <int kCachedVecs>
 __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __restrict__ x, int K, int ldx,
                                                              int8_t* __restrict__ xq, float* __restrict__ sx) {
   const int m = blockIdx.x;
@@ -62,7 +66,12 @@ __global__ void __launch_bounds__(kThreads) quant_act_kernel(const uint16_t* __r
 }  // namespace
 
 cudaError_t launch_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, cudaStream_t st) {
-  return launch_pdl(quant_act_kernel, dim3(M), dim3(kThreads), 0, st, x, K, ldx, xq, sx);
+  const int per_thread = (K / 8 + kThreads - 1) / kThreads;  // 16-byte vectors per thread
+  if (per_thread <= 1) return launch_pdl(quant_act_kernel<1>, dim3(M), dim3(kThreads), 0, st, x, K, ldx, xq, sx);
+  if (per_thread <= 2) return launch_pdl(quant_act_kernel<2>, dim3(M), dim3(kThreads), 0, st, x, K, ldx, xq, sx);
+  if (per_thread <= 4) return launch_pdl(quant_act_kernel<4>, dim3(M), dim3(kThreads), 0, st, x, K, ldx, xq, sx);
+  if (per_thread <= 8) return launch_pdl(quant_act_kernel<8>, dim3(M), dim3(kThreads), 0, st, x, K, ldx, xq, sx);
+  return launch_pdl(quant_act_kernel<kMaxCachedVecs>, dim3(M), dim3(kThreads), 0, st, x, K, ldx, xq, sx);
 }
 
 }  // namespace aq
