@@ -82,7 +82,7 @@ struct TcShape {
   static constexpr int kB = NT * kTileK;         // swizzled INT8 activation block
   static constexpr int kStageBytes = kA + kB + kStg;
   static constexpr int kStages = (200 * 1024) / kStageBytes < 8 ? (200 * 1024) / kStageBytes : 8;
-  static constexpr int kCols = NT <= 64 ? NT : 64;  // accumulator columns per epilogue thread
+  static constexpr int kCols = NT <= 64 ? NT : NT / 2;  // accumulator columns per epilogue thread
   static constexpr int kEpiWarps = 4 * NT / kCols;      // 4 warps (one per lane quadrant) per column group
   static constexpr int kThreads = 32 * kFirstEpiWarp + 32 * kEpiWarps;
   // Tensor-memory columns per load (one 16-column load; two register sets are
@@ -820,8 +820,21 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
   char* wsb = static_cast<char*>(ws);
   a.counters = reinterpret_cast<int*>(wsb + kWsHeader);
 
-  // token-block width: up to 64 tokens in one block of 16-multiples, 128 beyond
-  const int nt = M <= 64 ? (M + 15) / 16 * 16 : 128;
+  // token-block width: up to 64 tokens in one block of 16-multiples; beyond,
+  // 128 or 96 tokens, whichever leaves the shorter estimated makespan: whole
+  // units go to the CTAs in waves, and a 96-token tile costs about
+  // (128 + 96) / (128 + 128) of a 128-token one (half of a tile's time is
+  // fixed per tile), so 96 wins where it removes a mostly idle last wave
+  // (e.g. 2560 output features at 2048 tokens: 440 units in 3 waves instead
+  // of 320 in 3)
+  int nt = M <= 64 ? (M + 15) / 16 * 16 : 128;
+  if (M > 64) {
+    auto cost = [&](int t) {
+      const long long units = (long long)a.nrb * ((M + t - 1) / t);
+      return ((units + kNumSMs - 1) / kNumSMs) * (128 + t);
+    };
+    if (cost(96) < cost(128)) nt = 96;
+  }
   a.ntb = (M + nt - 1) / nt;
   if (phase == AQ_PHASE_DECODE && P == nullptr) {
     const DecodePlan p = plan_decode(M, w);
@@ -845,8 +858,14 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
     AQ_TC_CASE(32)
     AQ_TC_CASE(48)
     AQ_TC_CASE(64)
-    AQ_TC_CASE(128)
 #undef AQ_TC_CASE
+// more than 64 tokens: prefill only, never split
+#define AQ_TC_CASE_WIDE(NTV)                                             \
+  case NTV * 4 + 0: return launch_nt<NTV, 0>(w, xq, a, grid, st);      \
+  case NTV * 4 + 2: return launch_nt<NTV, 2>(w, xq, a, grid, st);
+    AQ_TC_CASE_WIDE(96)
+    AQ_TC_CASE_WIDE(128)
+#undef AQ_TC_CASE_WIDE
     default: return cudaErrorInvalidValue;
   }
 }
