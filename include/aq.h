@@ -211,6 +211,22 @@ int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, const float
                                void* stream);
 
 /*
+ * Activation quantization in the paper's own form (App. B.3; eq. 5, eq. 6 with
+ * b = 8), the activation side of its paper-exact numerics: one scale per
+ * group of 64 features and b_M rows, b_M = aq_act_group_rows(M) (1 for
+ * M = 1, else 16), rows zero-padded to M' = ceil(M / b_M) * b_M:
+ *   s = max(max(0, max A) / 127, max(0, -min A) / 128, 1e-12)   over group A
+ *   xq = clamp(rint(x / s), -128, 127) (fp64 quotient)            sx = (float)s
+ *  x   bf16 [M][ldx] device (bits as uint16), 16-byte aligned, ldx % 8 == 0, ldx >= K
+ *  xq  int8 [M'][K] device, 8-byte aligned; padding rows receive zero codes
+ *  sx  fp32 [M' / b_M][K / 64] device, row-major
+ * 1 <= M, 64 <= K <= 1048576 with K % 64 == 0.  Asynchronous on `stream`.
+ * Errors: AQ_ERR_ARG, AQ_ERR_CUDA.  aq_act_group_rows: host only, b_M (0 for M < 1).
+ */
+int aq_act_group_rows(int M);
+int aq_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream);
+
+/*
  * Device scratch bytes a linear call needs for `phase` (aq_phase) at M tokens
  * with packed weights *w (host struct; only its geometry is read).  Host only.
  * The workspace must be zero-filled once when allocated; afterwards the library

@@ -220,3 +220,16 @@ def test_long_prefill_sizes_and_validation():
     assert f(ctypes.byref(s), 16, 16, 300, None, 16, 0, 256, 16, ws, None, want, None) == -1
     assert f(ctypes.byref(s), 16, 16, 300, None, 16, 0, 256, 16, ws, 4096, want - 1, None) == -5
     assert f(ctypes.byref(s), 16, 16, 300, None, 16, 0, 256, 16, ws - 1, 4096, want, None) == -5
+
+
+def test_paper_form_activation_quantizer_validation():
+    L = aq.lib()
+    assert L.aq_act_group_rows(1) == 1 and L.aq_act_group_rows(2) == 16 and L.aq_act_group_rows(0) == 0
+    f = L.aq_quant_act_groups
+    assert f(None, 1, 128, 128, 16, 16, None) == -1
+    assert f(16, 0, 128, 128, 16, 16, None) == -1
+    assert f(16, 1, 96, 96, 16, 16, None) == -1       # K not a multiple of 64
+    assert f(16, 1, 128, 120, 16, 16, None) == -1     # ldx < K
+    assert f(16, 1, 128, 132, 16, 16, None) == -1     # ldx not a multiple of 8
+    assert f(24, 1, 128, 128, 16, 16, None) == -1     # x not 16-byte aligned
+    assert f(16, 1, 128, 128, 20, 16, None) == -1     # xq not 8-byte aligned

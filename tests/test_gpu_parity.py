@@ -434,3 +434,39 @@ def test_prefill_expanded_equals_prefill_bit_for_bit(M, bN, frac8, out_dtype):
     y2 = aq.aq_linear_prefill_expanded(w, xq, sx, bias=bias, out_dtype=out_dtype)
     assert torch.equal(y1, y2)
     assert_output_close(y2, oracle_linear(p, x, bias=bias.cpu().numpy()))
+
+
+# ------------------------------------------------------------------ paper-form activation quantization
+
+@pytest.mark.parametrize("M,K,pad,outlier", [(1, 64, 0, 0.0), (1, 3072, 8, 0.01), (2, 128, 0, 0.0),
+                                             (17, 2560, 0, 0.01), (300, 640, 16, 0.0), (2048, 2560, 0, 0.01)])
+def test_quant_act_groups_bit_exact(M, K, pad, outlier):
+    pn = oracle.aq_paper_numerics
+    x = synth.activations(M, K + pad, (M, K, pad, 7), outlier_frac=outlier)
+    if M > 2:
+        x[1, :64] = 0                                  # a zero row inside a group
+    if M >= 17:
+        x[16:, 64:128] = synth.f32_to_bf16_bits(-np.abs(oracle.bf16_bits_to_f64(x[16:, 64:128])).astype(np.float32))
+    xd = dev_bf16(x)
+    xq, sx = aq.aq_quant_act_groups(xd, K)
+    ref_q, ref_s, Mp = pn.quantize_activation_groups(oracle.bf16_bits_to_f64(x[:, :K]))
+    assert xq.shape == (Mp, K)
+    assert np.array_equal(xq.cpu().numpy(), ref_q)
+    assert np.array_equal(sx.cpu().numpy(), ref_s)
+
+
+def test_quant_act_groups_ties_and_endpoints():
+    # group scale 1 (max 127, min > -128): codes are rint of the values themselves;
+    # group scale 2 through the negative endpoint: -256 -> -128
+    pn = oracle.aq_paper_numerics
+    x = np.zeros((1, 128), np.float32)
+    x[0, :8] = [127.0, 2.5, -2.5, 3.5, 0.5, 1.5, -0.5, -127.0]
+    x[0, 64:70] = [-256.0, 5.0, 3.0, 1.0, -7.0, 100.0]
+    bits = synth.f32_to_bf16_bits(x)
+    xq, sx = aq.aq_quant_act_groups(dev_bf16(bits))
+    q = xq.cpu().numpy()
+    assert list(q[0, :8]) == [127, 2, -2, 4, 0, 2, 0, -127]
+    assert list(q[0, 64:70]) == [-128, 2, 2, 0, -4, 50]
+    assert list(sx.cpu().numpy()[0]) == [1.0, 2.0]
+    ref_q, ref_s, _ = pn.quantize_activation_groups(oracle.bf16_bits_to_f64(bits))
+    assert np.array_equal(q, ref_q) and np.array_equal(sx.cpu().numpy(), ref_s)

@@ -24,7 +24,7 @@ EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "
             "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
             "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc",
             "aq_quantize_weights", "aq_paper_packed_bytes", "aq_expanded_bytes", "aq_expand_int8",
-            "aq_linear_prefill_expanded")
+            "aq_linear_prefill_expanded", "aq_act_group_rows", "aq_quant_act_groups")
 
 
 class AqError(RuntimeError):
@@ -71,6 +71,10 @@ def lib():
     L.aq_linear_prefill_expanded.restype = c_int
     L.aq_linear_prefill_expanded.argtypes = [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p,
                                              c_size_t, c_void_p, c_size_t, c_void_p]
+    L.aq_act_group_rows.restype = c_int
+    L.aq_act_group_rows.argtypes = [c_int]
+    L.aq_quant_act_groups.restype = c_int
+    L.aq_quant_act_groups.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]
     L.aq_quantize_weights.restype = c_int
     L.aq_quantize_weights.argtypes = [c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_int,
                                       c_void_p, c_void_p, c_void_p]
@@ -219,6 +223,22 @@ def aq_quant_act(x: torch.Tensor, xq: torch.Tensor = None, sx: torch.Tensor = No
     _need(sx, "sx", torch.float32, x.device)
     _check(lib().aq_quant_act(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), sx.data_ptr(), _stream(x.device)),
            "aq_quant_act")
+    return xq, sx
+
+
+def aq_quant_act_groups(x: torch.Tensor, K: int = None):
+    """Paper-form activation quantization: x bf16 [M][ldx] -> (xq int8 [M'][K],
+    sx float32 [M'/b_M][K/64]) with one scale per 64 features x b_M rows."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor with unit inner stride")
+    M = x.shape[0]
+    K = x.shape[1] if K is None else K
+    bM = int(lib().aq_act_group_rows(M))
+    Mp = -(-M // bM) * bM
+    xq = torch.empty((Mp, K), dtype=torch.int8, device=x.device)
+    sx = torch.empty((Mp // bM, K // 64), dtype=torch.float32, device=x.device)
+    _check(lib().aq_quant_act_groups(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), sx.data_ptr(),
+                                     _stream(x.device)), "aq_quant_act_groups")
     return xq, sx
 
 

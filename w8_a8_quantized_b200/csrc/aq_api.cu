@@ -157,6 +157,21 @@ extern "C" int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const flo
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
 }
 
+namespace aq {
+int act_group_rows(int M);
+cudaError_t launch_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx,
+                                    cudaStream_t st);
+}  // namespace aq
+
+extern "C" int aq_act_group_rows(int M) { return M < 1 ? 0 : act_group_rows(M); }
+
+extern "C" int aq_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream) {
+  if (!x || !xq || !sx || M < 1 || K < 64 || K % 64 || K > (1 << 20) || ldx < K || ldx % 8) return AQ_ERR_ARG;
+  if (((uintptr_t)x & 15) || ((uintptr_t)xq & 7)) return AQ_ERR_ARG;
+  return launch_quant_act_groups(x, M, K, ldx, xq, sx, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? AQ_OK : AQ_ERR_CUDA;
+}
+
 extern "C" size_t aq_expanded_bytes(const aq_packed* w) {
   return validate_packed(w) == AQ_OK ? expanded_bytes(w) : 0;
 }
