@@ -289,6 +289,19 @@ class Model:
         return g, launches
 
 
+def max_over_ranks(torch, value: float, device) -> float:
+    """The largest of every rank's value; every rank calls it at the same point."""
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms: float, scale: float) -> float:
+    """Whole-job throughput: the units all ranks processed (each rank the same
+    amount: independent replicas) over the slowest rank's time, in units of `scale`."""
+    return world * units_per_rank / (ms * 1e-3) / scale
+
+
 def time_graph(torch, g, steps, warmup, dist_on, dev):
     for _ in range(warmup):
         g.replay()
@@ -308,9 +321,7 @@ def time_graph(torch, g, steps, warmup, dist_on, dev):
         torch.distributed.barrier()
     ms = e0.elapsed_time(e1) / steps
     if dist_on:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(torch, ms, dev)
     return ms
 
 
@@ -442,6 +453,8 @@ def main():
                 res.update(ms_e2e=float("nan"), h2d=0, d2h=0)
             else:
                 ms_e2e, h2d, d2h = time_e2e(torch, model, g, args.steps, args.warmup, dev)
+                if dist_on:  # every rank times it, the slowest one counts
+                    ms_e2e = max_over_ranks(torch, ms_e2e, dev)
                 res.update(ms_e2e=ms_e2e, h2d=h2d, d2h=d2h)
         results[M] = res
         aq.check_all_workspaces()
@@ -455,25 +468,25 @@ def main():
     wbytes = model.weight_bytes
     if decode:
         unit = "GB/s"
-        value = world * wbytes / (r0["ms"] * 1e-3) / 1e9
+        value = job_rate(world, wbytes, r0["ms"], 1e9)
         achieved = wbytes / (r0["ms_linear_only"] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": measured_traffic("decode"),
                 "algorithmic_bytes_per_launch": wbytes / r0["linear_launches"],
                 "kernel": "decode linear (all projections, activation quantization excluded)",
                 "peak_source": peaks["src"]}
-        e2e_val = world * wbytes / (r0["ms_e2e"] * 1e-3) / 1e9
+        e2e_val = job_rate(world, wbytes, r0["ms_e2e"], 1e9)
     else:
         unit = "TOPS"
         ops = 2.0 * model.M * model.macs
-        value = world * ops / (r0["ms"] * 1e-3) / 1e12
+        value = job_rate(world, ops, r0["ms"], 1e12)
         achieved = ops / (r0["ms_linear_only"] * 1e-3) / 1e12
         int8_peak = 2.0 * peaks["bf16"]  # dense INT8 = 2x dense BF16 (nominal ratio 4.5 / 2.25)
         roof = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TFLOP/s",
                 "frac": achieved / int8_peak, "traffic": measured_traffic("prefill"),
                 "kernel": "prefill linear (all projections, activation quantization excluded)",
                 "peak_source": f"{peaks['src']} bf16 x 2"}
-        e2e_val = world * ops / (r0["ms_e2e"] * 1e-3) / 1e12
+        e2e_val = job_rate(world, ops, r0["ms_e2e"], 1e12)
 
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,

@@ -1,0 +1,56 @@
+"""The multi-process (replica) path of the benchmark on CPU: two gloo ranks
+exercise the cross-rank reduction the benchmark uses (slowest rank's time)
+and the whole-job throughput (the units all ranks processed over that time).
+No GPU is involved."""
+import datetime
+import multiprocessing as mp
+import os
+import socket
+
+import pytest
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, times, q):
+    import torch
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        ms = bench.max_over_ranks(torch, times[rank], torch.device("cpu"))
+        q.put((rank, ms, bench.job_rate(world, 1.5e9, ms, 1e9)))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_replicas_report_slowest_rank_and_whole_job_rate(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    times = [2.0, 5.0, 3.0][:world]
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, times, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive and all(p.exitcode == 0 for p in procs)
+    out = sorted(q.get(timeout=5) for _ in range(world))
+    for rank, ms, rate in out:
+        assert ms == 5.0                                   # every rank sees the slowest time
+        assert rate == pytest.approx(world * 1.5 / 5e-3)   # world x 1.5 GB over 5 ms, in GB/s
+
+
+def test_job_rate_single_rank():
+    import bench
+    assert bench.job_rate(1, 2e12, 10.0, 1e12) == pytest.approx(200.0)
