@@ -55,12 +55,11 @@ WORKLOADS = {
                               outlier=0.01),
 }
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernels,
-# from the ncu captures summarised in profiles/, valid only while the kernel source is unchanged
+# from an ncu capture of the named workload, valid only while the kernel source is unchanged
 # (sha256 prefix of the source file and the shared header).
 MEASURED_TRAFFIC = {
-    # profiles/decode_rows_llama3b_1token.md: one layer's four launches read 64,740,608 B and wrote
-    # 23,808 B -> 16,191,104 B per launch (algorithmic: 16,128,638 B per launch); the hash covers the
-    # shared header too, which has since gained host-side declarations only
+    # one Llama-3.2-3B layer's four decode launches at 1 token read 64,740,608 B and wrote
+    # 23,808 B -> 16,191,104 B per launch (algorithmic: 16,128,638 B per launch)
     "decode": {"src": ("w8_a8_quantized_b200/csrc/decode_rows.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
                "sha": "9ff17c3bbdb451a8", "bytes_per_launch": 16191104},
     "prefill": {"src": ("w8_a8_quantized_b200/csrc/tc_linear.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),

@@ -171,11 +171,33 @@ def aq_pack(codes: torch.Tensor, scales: torch.Tensor, pmap: torch.Tensor, bN: i
     _need(scales, "scales", torch.float16, dev)
     _need(pmap, "pmap", torch.uint8, dev)
     N, K = codes.shape
-    T4 = int(pmap.sum().item())
+    T4 = aq_int4_tiles(pmap)
+    if scales.dim() != 2 or scales.shape[0] != N or pmap.dim() != 2 or pmap.shape[0] * bN != N or \
+            pmap.shape[1] * bK != K or scales.shape[1] != pmap.shape[1]:
+        raise ValueError("codes [N][K], scales [N][C] and pmap [R][C] do not agree with the tile shape")
     w = PackedWeights(N, K, bN, bK, T4, dev)
-    _check(lib().aq_pack(codes.data_ptr(), scales.data_ptr(), pmap.data_ptr(), N, K, bN, bK,
-                         ctypes.byref(w.struct), _stream(dev)), "aq_pack")
+    with torch.cuda.device(dev):
+        _check(lib().aq_pack(codes.data_ptr(), scales.data_ptr(), pmap.data_ptr(), N, K, bN, bK,
+                             ctypes.byref(w.struct), _stream(dev)), "aq_pack")
     return w
+
+
+def aq_int4_tiles(pmap: torch.Tensor) -> int:
+    """INT4 tile count of a precision map (uint8 [R][C], 1 = INT4), as the library's
+    host-side metadata builder counts it; it rejects labels other than 0 and 1."""
+    if pmap.dim() != 2 or pmap.dtype != torch.uint8:
+        raise ValueError("pmap must be a 2-D uint8 tensor")
+    R, C = pmap.shape
+    host = np.ascontiguousarray(pmap.cpu().numpy())
+    T = R * C
+    bitmap = np.zeros(max((T + 7) // 8, 1), np.uint8)
+    off4, off8 = np.zeros(R + 1, np.int32), np.zeros(R + 1, np.int32)
+    idx = np.zeros(max(T, 1), np.int32)
+    t4 = ctypes.c_int32(0)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().aq_pack_metadata(p(host), R, C, p(bitmap), p(off4), p(off8), p(idx), ctypes.byref(t4)),
+           "aq_pack_metadata")
+    return int(t4.value)
 
 
 def aq_quantize_weights(w: torch.Tensor, pmap: torch.Tensor, bN: int, bK: int = 128, search: bool = True,
@@ -221,8 +243,11 @@ def aq_quant_act(x: torch.Tensor, xq: torch.Tensor = None, sx: torch.Tensor = No
         sx = torch.empty((M,), dtype=torch.float32, device=x.device)
     _need(xq, "xq", torch.int8, x.device)
     _need(sx, "sx", torch.float32, x.device)
-    _check(lib().aq_quant_act(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), sx.data_ptr(), _stream(x.device)),
-           "aq_quant_act")
+    if xq.dim() != 2 or xq.shape[0] < M or xq.shape[1] != K or sx.numel() < M or x.shape[1] < K:
+        raise ValueError("xq must be [M][K] and sx hold M scales, with K <= x.shape[1]")
+    with torch.cuda.device(x.device):
+        _check(lib().aq_quant_act(x.data_ptr(), M, K, x.stride(0), xq.data_ptr(), sx.data_ptr(),
+                                  _stream(x.device)), "aq_quant_act")
     return xq, sx
 
 
@@ -262,22 +287,39 @@ def workspace(phase: int, M: int, w: PackedWeights) -> torch.Tensor:
     return ws
 
 
-def _linear(fn, name, phase, w, xq, sx, bias, out, out_dtype, ws):
+def _linear_operands(w, xq, sx, bias, out, out_dtype):
+    """Check the operands of a linear call against the packed weights (shapes the
+    kernels read and write through raw pointers); allocate `out` if absent."""
     _need(xq, "xq", torch.int8, w.device)
     _need(sx, "sx", torch.float32, w.device)
+    if xq.dim() != 2 or xq.shape[1] != w.K:
+        raise ValueError(f"xq must be [M][{w.K}], got {tuple(xq.shape)}")
     M = xq.shape[0]
+    if M < 1 or sx.numel() < M:
+        raise ValueError(f"sx must hold at least M = {M} token scales")
     if out is None:
         out = torch.empty((M, w.N), dtype=out_dtype, device=w.device)
-    if out.dtype not in (torch.float32, torch.bfloat16) or out.stride(1) != 1 or out.device != w.device:
-        raise ValueError("out must be float32 or bfloat16 on the weights' device with unit inner stride")
-    ydt = AQ_F32 if out.dtype == torch.float32 else AQ_BF16
+    if out.dtype not in (torch.float32, torch.bfloat16) or out.dim() != 2 or out.stride(1) != 1 or \
+            out.device != w.device:
+        raise ValueError("out must be a 2-D float32 or bfloat16 tensor on the weights' device, unit inner stride")
+    if out.shape[0] < M or out.shape[1] < w.N:
+        raise ValueError(f"out must be at least [{M}][{w.N}], got {tuple(out.shape)}")
     if bias is not None:
         _need(bias, "bias", torch.float32, w.device)
+        if bias.numel() < w.N:
+            raise ValueError(f"bias must hold N = {w.N} values")
+    return M, out
+
+
+def _linear(fn, name, phase, w, xq, sx, bias, out, out_dtype, ws):
+    M, out = _linear_operands(w, xq, sx, bias, out, out_dtype)
+    ydt = AQ_F32 if out.dtype == torch.float32 else AQ_BF16
     if ws is None:
         ws = workspace(phase, M, w)
-    _check(fn(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
-              bias.data_ptr() if bias is not None else None, out.data_ptr(), ydt, out.stride(0),
-              ws.data_ptr(), ws.numel(), _stream(w.device)), name)
+    with torch.cuda.device(w.device):
+        _check(fn(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
+                  bias.data_ptr() if bias is not None else None, out.data_ptr(), ydt, out.stride(0),
+                  ws.data_ptr(), ws.numel(), _stream(w.device)), name)
     return out
 
 
@@ -354,19 +396,13 @@ def aq_linear_decode_noalloc(w: PackedWeights, xq, sx, bias=None, out=None, out_
     memory: the library's fixed 4 MiB device scratch is used instead (calls that
     overlap on the GPU must not share it).  `out` must be preallocated by callers
     that cannot allocate; it is allocated here only for convenience."""
-    _need(xq, "xq", torch.int8, w.device)
-    _need(sx, "sx", torch.float32, w.device)
-    M = xq.shape[0]
-    if out is None:
-        out = torch.empty((M, w.N), dtype=out_dtype, device=w.device)
-    if out.dtype not in (torch.float32, torch.bfloat16) or out.stride(1) != 1 or out.device != w.device:
-        raise ValueError("out must be float32 or bfloat16 on the weights' device with unit inner stride")
-    if bias is not None:
-        _need(bias, "bias", torch.float32, w.device)
-    _check(lib().aq_linear_decode_noalloc(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
-                                          bias.data_ptr() if bias is not None else None, out.data_ptr(),
-                                          AQ_F32 if out.dtype == torch.float32 else AQ_BF16, out.stride(0),
-                                          _stream(w.device)), "aq_linear_decode_noalloc")
+    M, out = _linear_operands(w, xq, sx, bias, out, out_dtype)
+    # the library resolves its scratch array on the CURRENT device: make it the weights' device
+    with torch.cuda.device(w.device):
+        _check(lib().aq_linear_decode_noalloc(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
+                                              bias.data_ptr() if bias is not None else None, out.data_ptr(),
+                                              AQ_F32 if out.dtype == torch.float32 else AQ_BF16, out.stride(0),
+                                              _stream(w.device)), "aq_linear_decode_noalloc")
     return out
 
 
@@ -390,8 +426,15 @@ class Group:
         dev = self.weights[0].device
         if x.dtype != torch.bfloat16 or x.device != dev or x.dim() != 2 or x.stride(1) != 1:
             raise ValueError("x must be a 2-D bf16 tensor on the weights' device with unit inner stride")
-        if x.shape[0] != self.M or len(outs) != G:
-            raise ValueError("token count or number of outputs does not match the group")
+        if x.shape[0] != self.M or x.shape[1] < self.weights[0].K or len(outs) != G:
+            raise ValueError("token count, input width or number of outputs does not match the group")
+        for o, w in zip(outs, self.weights):
+            if o.dim() != 2 or o.shape[0] < self.M or o.shape[1] < w.N:
+                raise ValueError(f"each output must be at least [M][N] = [{self.M}][{w.N}]")
+        if bias is not None and (len(bias) != G or any(b is not None and (b.dtype != torch.float32 or
+                                                                       b.device != dev or b.numel() < w.N)
+                                                      for b, w in zip(bias, self.weights))):
+            raise ValueError("bias must hold one float32 [N] tensor (or None) per member")
         dt = outs[0].dtype
         if dt not in (torch.float32, torch.bfloat16) or any(o.dtype != dt or o.device != dev or o.stride(1) != 1
                                                              for o in outs):
@@ -402,21 +445,25 @@ class Group:
         if bias is not None:
             bs = (ctypes.c_void_p * G)(*[b.data_ptr() if b is not None else None for b in bias])
         ws = self.ws if ws is None else ws
-        _check(lib().aq_linear_group(self.phase, self._w, G, x.data_ptr(), x.stride(0), self.M, bs, ys, lds,
-                                     AQ_F32 if dt == torch.float32 else AQ_BF16, ws.data_ptr(), ws.numel(),
-                                     _stream(dev)), "aq_linear_group")
+        with torch.cuda.device(dev):
+            _check(lib().aq_linear_group(self.phase, self._w, G, x.data_ptr(), x.stride(0), self.M, bs, ys, lds,
+                                         AQ_F32 if dt == torch.float32 else AQ_BF16, ws.data_ptr(), ws.numel(),
+                                         _stream(dev)), "aq_linear_group")
         return outs
 
 
 def aq_debug_tile_partials(w: PackedWeights, xq: torch.Tensor, phase: int, ws=None) -> torch.Tensor:
     """Exact INT32 tile products P[M][N][C] computed by the `phase` data path."""
     _need(xq, "xq", torch.int8, w.device)
+    if xq.dim() != 2 or xq.shape[1] != w.K:
+        raise ValueError(f"xq must be [M][{w.K}]")
     M = xq.shape[0]
     P = torch.zeros((M, w.N, w.C), dtype=torch.int32, device=w.device)
     if ws is None:
         ws = workspace(AQ_PHASE_PREFILL, M, w)
-    _check(lib().aq_debug_tile_partials(ctypes.byref(w.struct), xq.data_ptr(), M, phase, P.data_ptr(),
-                                        ws.data_ptr(), ws.numel(), _stream(w.device)), "aq_debug_tile_partials")
+    with torch.cuda.device(w.device):
+        _check(lib().aq_debug_tile_partials(ctypes.byref(w.struct), xq.data_ptr(), M, phase, P.data_ptr(),
+                                            ws.data_ptr(), ws.numel(), _stream(w.device)), "aq_debug_tile_partials")
     return P
 
 

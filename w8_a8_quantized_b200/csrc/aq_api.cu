@@ -3,10 +3,38 @@
 // arguments, enqueues its kernels on the caller's stream and returns without
 // allocating or synchronizing.
 #include <algorithm>
+#include <atomic>
 
 #include "aq_internal.cuh"
 
 namespace aq {
+
+int num_sms() {
+  static std::atomic<int> cached[kMaxDevices];
+  constexpr int kFallback = 148;  // B200
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return kFallback;
+  }
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+    cudaGetLastError();
+    return kFallback;
+  }
+  cached[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+bool set_smem_attr_once(const void* kernel, int bytes, std::atomic<bool>* done_flags) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (done_flags[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done_flags[dev].store(true, std::memory_order_release);
+  return true;
+}
 
 int validate_packed(const aq_packed* w) {
   if (!w) return AQ_ERR_ARG;
@@ -39,8 +67,8 @@ DecodePlan plan_decode(int M, const aq_packed* w) {
   DecodePlan p;
   if (rows_supported(M, w->K) && M <= kRowsPreferM) {
     p.kernel = 0;
-    p.rows = 16;
-    p.blocks = w->N / 16;
+    p.rows = kRowsPerCta;
+    p.blocks = w->N / kRowsPerCta;
     p.S = 1;
   } else {
     p.kernel = 1;
@@ -48,7 +76,7 @@ DecodePlan plan_decode(int M, const aq_packed* w) {
     p.blocks = ceil_div(w->R, 128 / w->bN);
     // one wave (blocks x S <= SMs), and at most kMaxSplits: the CTA that sums a
     // unit's splits pays one round of L2 latency per split
-    p.S = std::max(1, std::min(std::min(w->C, kMaxSplits), kNumSMs / p.blocks));
+    p.S = std::max(1, std::min(std::min(w->C, kMaxSplits), num_sms() / p.blocks));
   }
   return p;
 }
@@ -68,7 +96,7 @@ size_t prefill_ws_bytes(int /*M*/, const aq_packed* w) { return kWsHeader + coun
 DecodeProj decode_proj(const aq_packed* w, const float* bias, void* y, int ldy) {
   DecodeProj d;
   d.bitmap = w->bitmap; d.tile_idx = w->tile_idx; d.w4 = w->w4; d.w8 = w->w8; d.scales = w->scales;
-  d.bias = bias; d.y = y; d.N = w->N; d.bN = w->bN; d.ldy = ldy; d.blocks = w->N / 16;
+  d.bias = bias; d.y = y; d.N = w->N; d.bN = w->bN; d.ldy = ldy; d.blocks = w->N / kRowsPerCta;
   return d;
 }
 
@@ -319,12 +347,14 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
 extern "C" int aq_workspace_status(void* ws, void* stream, int* info) {
   if (!ws) return AQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  WsHeader h{0, 0};
+  WsHeader h{0, 0, 0};
   if (cudaStreamSynchronize(st) != cudaSuccess) return AQ_ERR_CUDA;
   if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return AQ_ERR_CUDA;
   if (h.err_code != 0) {
-    const WsHeader zero{0, 0};
-    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return AQ_ERR_CUDA;
+    // a call that gave up may have left split-K arrival counters nonzero: the
+    // kernel recorded how many bytes after the header to zero with the error
+    const size_t clear = kWsHeader + (size_t)std::max(h.err_clear, 0);
+    if (cudaMemset(ws, 0, clear) != cudaSuccess) return AQ_ERR_CUDA;
   }
   if (info) *info = h.err_info;
   return h.err_code == 0 ? AQ_OK : AQ_ERR_TIMEOUT;

@@ -10,14 +10,21 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/aq.h"
 
 namespace aq {
 
 // ---------------------------------------------------------------- geometry
 constexpr int kTileK = 128;          // bK: the only supported input-tile width
-constexpr int kNumSMs = 148;         // B200; used to size split counts on the host
 constexpr int kMaxDecodeM = 64;
+constexpr int kMaxDevices = 64;      // per-device host caches
+
+// Streaming multiprocessors of the current device (cached per device; 148 on a
+// B200, also the answer when no device can be queried, e.g. for host-only
+// sizing calls on a machine without a GPU).  Sizes grids and split counts.
+int num_sms();
 
 // Workspace layout.  The first 256 bytes hold the error word; split-K
 // counters and fp32 partial sums follow.
@@ -25,6 +32,7 @@ constexpr size_t kWsHeader = 256;
 struct WsHeader {
   int err_code;   // 0 or AQ_ERR_TIMEOUT
   int err_info;   // which wait gave up (kernel-specific code)
+  int err_clear;  // bytes after the header (split-K counters) to zero again after an error
 };
 
 // Bounded waits: any spin on an mbarrier gives up after this long, records
@@ -41,6 +49,7 @@ int validate_packed(const aq_packed* w);  // AQ_OK or an error status
 // One projection as seen by the CUDA-core decode kernel (a group of up to
 // kMaxGroup projections sharing one input runs as a single launch).
 constexpr int kMaxGroup = 3;
+constexpr int kRowsPerCta = 32;                // output rows per CTA of the CUDA-core decode kernel
 constexpr int kRowsMaxM = 8;                   // tokens handled by the CUDA-core decode kernel
 constexpr size_t kFusedMaxBytes = 64 * 1024;   // shared memory for fused activation codes
 struct DecodeProj {
@@ -64,8 +73,8 @@ cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint
 struct DecodePlan {
   int kernel;   // 0 = CUDA-core kernel, 1 = tensor-core kernel
   int S;        // splits over tile columns
-  int rows;     // output rows per CTA block (128 or 64)
-  int blocks;   // number of row blocks
+  int rows;     // output rows per CTA (kRowsPerCta, or 128 for the tensor-core kernel)
+  int blocks;   // number of CTA row blocks
 };
 DecodePlan plan_decode(int M, const aq_packed* w);
 size_t decode_ws_bytes(int M, const aq_packed* w);
@@ -256,9 +265,15 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-__device__ __forceinline__ void record_error(void* ws, int code, int info) {
+// Records the first error of a launch.  `clear_bytes`: the bytes after the
+// header (split-K arrival counters) that a call which gave up may have left
+// nonzero; the status call zeroes them so the workspace is ready again.
+__device__ __forceinline__ void record_error(void* ws, int code, int info, int clear_bytes) {
   WsHeader* h = reinterpret_cast<WsHeader*>(ws);
-  if (atomicCAS(&h->err_code, 0, code) == 0) atomicExch(&h->err_info, info);
+  if (atomicCAS(&h->err_code, 0, code) == 0) {
+    atomicExch(&h->err_info, info);
+    atomicExch(&h->err_clear, clear_bytes);
+  }
 }
 
 // Programmatic dependent launch controls (no-ops without the launch attribute).
@@ -281,10 +296,13 @@ __device__ __forceinline__ float abs_max8(const uint4& v, float m) {
 }
 
 // s = max(fl64(amax / 127), 1e-12) (eq. 6 floor).  The quotient is formed from
-// the rounded reciprocal R = fl64(1/127) and one exact residual correction:
-// q = amax R, r = fma(-q, 127, amax) (exact), s = fma(r, R, q).  For every
-// finite bf16 amax this equals the IEEE fp64 quotient (checked exhaustively),
-// at a fraction of a division's latency.
+// the rounded reciprocal R = fl64(1/127) and one exact residual correction
+// (the FMA-based quotient correction of P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Develop. 34(1), 1990): q = amax R, r = fma(-q, 127, amax) (exact),
+// s = fma(r, R, q).  For every finite bf16 amax this equals the IEEE fp64
+// quotient (checked exhaustively against the oracle's division), at a
+// fraction of a division's latency.
 __device__ __forceinline__ double act_scale(float amax) {
   constexpr double kInv127 = 1.0 / 127.0;
   const double a = static_cast<double>(amax);
@@ -358,6 +376,17 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Opt a kernel in to `bytes` of dynamic shared memory on the current device.
+// The attribute is per device, so it is set once per (kernel, device); the
+// flags are atomics, so concurrent host threads at worst set it twice.
+bool set_smem_attr_once(const void* kernel, int bytes, std::atomic<bool>* done_flags);
+template <auto Kernel>
+cudaError_t ensure_smem_attr(int bytes) {
+  static std::atomic<bool> done[kMaxDevices];
+  return set_smem_attr_once(reinterpret_cast<const void*>(Kernel), bytes, done) ? cudaSuccess
+                                                                               : cudaErrorInvalidValue;
 }
 
 }  // namespace aq

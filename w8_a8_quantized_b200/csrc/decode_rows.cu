@@ -44,7 +44,7 @@
 namespace aq {
 namespace {
 
-constexpr int kRows = 32;
+constexpr int kRows = kRowsPerCta;
 constexpr int kGroupThreads = kRows * 2;  // threads of one tile group
 constexpr int kMaxKG = 8;
 constexpr int kMaxThreads = kGroupThreads * kMaxKG;
@@ -355,13 +355,8 @@ __global__ void __launch_bounds__(kMaxThreads) decode_rows_kernel(const __grid_c
 
 template <int MT, bool FUSED, bool DEBUG>
 cudaError_t launch_rows_t(const RowsArgs& a, int blocks, size_t smem, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(decode_rows_kernel<MT, FUSED, DEBUG>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFusedMaxBytes);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  cudaError_t e = ensure_smem_attr<decode_rows_kernel<MT, FUSED, DEBUG>>((int)kFusedMaxBytes);
+  if (e != cudaSuccess) return e;
   return launch_pdl(decode_rows_kernel<MT, FUSED, DEBUG>, dim3(blocks), dim3(kGroupThreads * a.KG), smem, st, a);
 }
 
@@ -394,9 +389,10 @@ cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint
   // at most 256 threads (room for the next launch's CTAs) unless rows are long
   // or the launch has no more CTAs than SMs (then wider CTAs only shorten the
   // per-thread tile loop; with more CTAs 512-thread CTAs would need a second wave)
-  const int kg_cap = (a.C >= 32 || blocks <= kNumSMs) ? kMaxKG : 4;
+  const int sms = num_sms();
+  const int kg_cap = (a.C >= 32 || blocks <= sms) ? kMaxKG : 4;
   int KG = 1;
-  while (KG < kg_cap && warps * KG < 16 * kNumSMs && a.C >= 4 * KG) KG *= 2;
+  while (KG < kg_cap && warps * KG < 16 * sms && a.C >= 4 * KG) KG *= 2;
   a.KG = KG;
   if (P != nullptr) return launch_rows_m<false, true>(a, blocks, 0, st);
   if (x != nullptr) return launch_rows_m<true, false>(a, blocks, 2 * (size_t)M * K + 16 * (size_t)M, st);

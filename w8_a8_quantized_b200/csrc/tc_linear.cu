@@ -137,6 +137,7 @@ struct TcArgs {
   void* ws;
   float* partial;  // [S][N][Mp], Mp = M rounded up to a multiple of 4
   int* counters;   // [nrb * ntb]
+  int ws_clear;    // bytes of split-K counters after the workspace header (0 without splits)
   int32_t* P;      // debug: exact tile products [M][N][C], or null
 };
 
@@ -383,7 +384,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
 
   auto fail = [&](int info) {
     *abort_flag = 1;
-    record_error(a.ws, AQ_ERR_TIMEOUT, info);
+    record_error(a.ws, AQ_ERR_TIMEOUT, info, a.ws_clear);
   };
 
   if (warp == 0) {
@@ -786,13 +787,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
 template <int NT, int MODE>
 cudaError_t launch_nt(const aq_packed* w, const int8_t* xq, TcArgs a, int grid, cudaStream_t st) {
   using Sh = TcShape<NT>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(tc_linear_kernel<NT, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Sh::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_smem_attr<tc_linear_kernel<NT, MODE>>(Sh::kSmemBytes);
+  if (e != cudaSuccess) return e;
   CUtensorMap m8, m4, mx;
   memset(&m8, 0, sizeof(m8));
   memset(&m4, 0, sizeof(m4));
@@ -827,11 +823,12 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
   // fixed per tile), so 96 wins where it removes a mostly idle last wave
   // (e.g. 2560 output features at 2048 tokens: 440 units in 3 waves instead
   // of 320 in 3)
+  const int sms = num_sms();
   int nt = M <= 64 ? (M + 15) / 16 * 16 : 128;
   if (M > 64) {
     auto cost = [&](int t) {
       const long long units = (long long)a.nrb * ((M + t - 1) / t);
-      return ((units + kNumSMs - 1) / kNumSMs) * (128 + t);
+      return ((units + sms - 1) / sms) * (128 + t);
     };
     if (cost(96) < cost(128)) nt = 96;
   }
@@ -842,12 +839,14 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
     if (a.S > kMaxTcSplits) return cudaErrorInvalidValue;  // the split reduction unrolls over kMaxTcSplits
     const size_t cnt_bytes = ((size_t)p.blocks * sizeof(int) + 255) / 256 * 256;
     a.partial = reinterpret_cast<float*>(wsb + kWsHeader + cnt_bytes);
+    a.ws_clear = a.S > 1 ? (int)cnt_bytes : 0;
   } else {
     a.S = 1;
     a.partial = nullptr;
+    a.ws_clear = 0;
   }
   a.units = a.nrb * a.ntb * a.S;
-  const int grid = std::min(a.units, kNumSMs);
+  const int grid = std::min(a.units, sms);
   const int mode = P ? 2 : (a.S > 1 ? 1 : 0);
   switch (nt * 4 + mode) {
 #define AQ_TC_CASE(NTV)                                                  \
