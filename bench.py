@@ -253,21 +253,21 @@ class Model:
         expanded to a temporary INT8 copy, then the pure INT8 GEMM)."""
         aq = self.aq
         n = 0
-        for l in range(self.layers):
-            for kind, names in self.members.items():
-                if mode == "group":
-                    self.groups[l][kind](self.x[l][kind], [self.y[nm] for nm in names], ws=self.ws)
-                    rows = self.phase == aq.AQ_PHASE_DECODE and (self.M <= 4 or (len(names) >= 3 and self.M <= 8))
-                    n += 1 if self.fused else 1 + (1 if rows else len(names))  # fused, or quantize + members
-                elif mode == "expanded":
-                    for nm in names:
-                        aq.aq_linear_prefill_expanded(self.weights[l][nm], self.xq[kind], self.sx[kind],
-                                                      out=self.y[nm], ws=self.ws, tmp=self.tmp)
-                        n += 2
-                else:
-                    for nm in names:
-                        self.run(self.weights[l][nm], self.xq[kind], self.sx[kind], out=self.y[nm], ws=self.ws)
-                        n += 1
+        for l, kind in [(l, kind) for l in range(self.layers) for kind in self.members]:
+            names = self.members[kind]
+            if mode == "group":
+                self.groups[l][kind](self.x[l][kind], [self.y[nm] for nm in names], ws=self.ws)
+                rows = self.phase == aq.AQ_PHASE_DECODE and (self.M <= 4 or (len(names) >= 3 and self.M <= 8))
+                n += 1 if self.fused else 1 + (1 if rows else len(names))  # fused, or quantize + members
+            elif mode == "expanded":
+                for nm in names:
+                    aq.aq_linear_prefill_expanded(self.weights[l][nm], self.xq[kind], self.sx[kind],
+                                                  out=self.y[nm], ws=self.ws, tmp=self.tmp)
+                    n += 2
+            else:
+                for nm in names:
+                    self.run(self.weights[l][nm], self.xq[kind], self.sx[kind], out=self.y[nm], ws=self.ws)
+                    n += 1
         return n
 
     def quantize_inputs(self):

@@ -207,6 +207,35 @@ def _group_case(shapes, M, seed, phase, bN=128, frac8=0.25):
     return ps, ws, x
 
 
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("N,K,bN", [(256, 6144, 128), (384, 5120, 64), (1536, 4096, 128)])
+def test_decode_long_rows_reuse_every_ring_slot(M, N, K, bN):
+    """Few rows per CTA and long rows: every CTA of the streaming decode kernel
+    walks many more stages than its ring has slots (each slot is refilled several
+    times, across row blocks), so the ring's phase bookkeeping is exercised.
+    Outputs against the oracle, per-tile products bit-exact."""
+    p, x, w, xq, sx = packed_case(N, K, bN, 0.3, 1400 + M + N, M, outlier=0.01)
+    assert_output_close(aq.aq_linear_decode(w, xq, sx), oracle_linear(p, x))
+    P = aq.aq_debug_tile_partials(w, xq, aq.AQ_PHASE_DECODE)
+    assert np.array_equal(P.cpu().numpy(), oracle.tile_partials(p.codes, oracle.quant_act(x)[0], 128))
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_group_fused_long_rows(M):
+    """A fused q/k/v-style group whose CTAs each stream several row blocks of 40
+    tile columns (ring slots refilled many times)."""
+    shapes = [(1024, 5120), (256, 5120), (256, 5120)]
+    ps, ws, x = _group_case(shapes, M, 1500 + M, aq.AQ_PHASE_DECODE)
+    grp = aq.Group(ws, aq.AQ_PHASE_DECODE, M)
+    outs = [torch.empty((M, N), device="cuda") for N, _ in shapes]
+    for _ in range(3):  # repeated calls reuse the same graph of barriers from a clean start
+        grp(dev_bf16(x), outs)
+    for p, o in zip(ps, outs):
+        assert_output_close(o, oracle_linear(p, x))
+    rc, _ = aq.aq_workspace_status(grp.ws)
+    assert rc == 0
+
+
 @pytest.mark.parametrize("M", [1, 3, 8])
 def test_decode_wide_layer_matches_oracle(M):
     """A layer wider than one 32-row CUDA-core block per SM (so blocks queue

@@ -445,10 +445,10 @@ class Group:
         if bias is not None:
             bs = (ctypes.c_void_p * G)(*[b.data_ptr() if b is not None else None for b in bias])
         ws = self.ws if ws is None else ws
+        ydt = AQ_F32 if dt == torch.float32 else AQ_BF16
         with torch.cuda.device(dev):
             _check(lib().aq_linear_group(self.phase, self._w, G, x.data_ptr(), x.stride(0), self.M, bs, ys, lds,
-                                         AQ_F32 if dt == torch.float32 else AQ_BF16, ws.data_ptr(), ws.numel(),
-                                         _stream(dev)), "aq_linear_group")
+                                         ydt, ws.data_ptr(), ws.numel(), _stream(dev)), "aq_linear_group")
         return outs
 
 

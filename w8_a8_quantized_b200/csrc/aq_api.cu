@@ -27,13 +27,34 @@ int num_sms() {
   return v;
 }
 
-bool set_smem_attr_once(const void* kernel, int bytes, std::atomic<bool>* done_flags) {
+bool set_smem_attr_once(const void* kernel, int bytes, int carveout_pct, std::atomic<bool>* done_flags) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (done_flags[dev].load(std::memory_order_acquire)) return true;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (carveout_pct >= 0 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, carveout_pct) != cudaSuccess)
+    return false;
   done_flags[dev].store(true, std::memory_order_release);
   return true;
+}
+
+// The streaming kernel takes one token; from two tokens on the register-ring
+// kernel measured faster on the benchmark's decode step (1.36 against 1.55 ms
+// per Llama-3.2-3B step at 2 tokens), and they tie at 4.
+static constexpr int kStreamMaxM = 1;
+
+bool cc_fusable(int M, int K, int rows) {
+  return (M <= kStreamMaxM && stream_supported(M, K, rows)) || rows_fusable(M, K);
+}
+
+cudaError_t launch_decode_cc(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
+                             const float* sx, int M, int ydtype, int32_t* P, void* ws, cudaStream_t st) {
+  int rows = 0;
+  for (int g = 0; g < G; ++g) rows += projs[g].N;
+  if (M <= kStreamMaxM && stream_supported(M, K, rows))
+    return launch_decode_stream(projs, G, K, x, ldx, xq, sx, M, ydtype, P, ws, st);
+  return launch_decode_rows(projs, G, K, x, ldx, xq, sx, M, ydtype, P, ws, st);
 }
 
 int validate_packed(const aq_packed* w) {
@@ -168,7 +189,7 @@ extern "C" int aq_linear_decode(const aq_packed* w, const int8_t* xq, const floa
   cudaError_t e;
   if (plan_decode(M, w).kernel == 0) {
     const DecodeProj d = decode_proj(w, bias, y, ldy);
-    e = launch_decode_rows(&d, 1, w->K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+    e = launch_decode_cc(&d, 1, w->K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
   } else {
     e = launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_DECODE, st);
   }
@@ -223,7 +244,8 @@ extern "C" int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   aq_packed e;
   cudaError_t err = launch_expand_int8(w, tmp, &e, st);
-  if (err == cudaSuccess) err = launch_tc(&e, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_PREFILL, st);
+  if (err == cudaSuccess)
+    err = launch_tc(&e, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_PREFILL, st);
   return err == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
 }
 
@@ -239,7 +261,7 @@ extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int 
   cudaError_t e;
   if (phase == AQ_PHASE_DECODE && plan_decode(M, w).kernel == 0) {
     const DecodeProj d = decode_proj(w, nullptr, nullptr, w->N);
-    e = launch_decode_rows(&d, 1, w->K, nullptr, 0, xq, nullptr, M, AQ_F32, P, ws, st);
+    e = launch_decode_cc(&d, 1, w->K, nullptr, 0, xq, nullptr, M, AQ_F32, P, ws, st);
   } else
     e = launch_tc(w, xq, nullptr, M, nullptr, nullptr, AQ_F32, w->N, ws, P, phase, st);
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
@@ -261,8 +283,10 @@ static int check_group(int phase, const aq_packed* const* w, int G, const uint16
 }
 
 static bool group_fused(int phase, const aq_packed* const* w, int G, int M) {
-  return phase == AQ_PHASE_DECODE && rows_supported(M, w[0]->K) && rows_fusable(M, w[0]->K);
-  (void)G;
+  if (phase != AQ_PHASE_DECODE || !rows_supported(M, w[0]->K)) return false;
+  int rows = 0;
+  for (int g = 0; g < G; ++g) rows += w[g]->N;
+  return cc_fusable(M, w[0]->K, rows);
 }
 
 static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
@@ -314,7 +338,7 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   if (group_fused(phase, w, G, M)) {
     DecodeProj d[kMaxGroup];
     for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
-    e = launch_decode_rows(d, G, K, x, ldx, nullptr, nullptr, M, ydtype, nullptr, ws, st);
+    e = launch_decode_cc(d, G, K, x, ldx, nullptr, nullptr, M, ydtype, nullptr, ws, st);
     return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
   }
   // prepare the shared input once, then run the members on it (one launch
@@ -329,14 +353,14 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   if (e == cudaSuccess && group_rows(phase, w, G, M)) {  // one CUDA-core launch over all members' rows
     DecodeProj d[kMaxGroup];
     for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
-    e = launch_decode_rows(d, G, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+    e = launch_decode_cc(d, G, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
     return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
   }
   for (int g = 0; e == cudaSuccess && g < G; ++g) {
     const float* b = bias ? bias[g] : nullptr;
     if (phase == AQ_PHASE_DECODE && plan_decode(M, w[g]).kernel == 0) {
       const DecodeProj d = decode_proj(w[g], b, y[g], ldy[g]);
-      e = launch_decode_rows(&d, 1, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+      e = launch_decode_cc(&d, 1, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
     } else {
       e = launch_tc(w[g], xq, sx, M, b, y[g], ydtype, ldy[g], ws, nullptr, phase, st);
     }

@@ -66,7 +66,21 @@ DecodeProj decode_proj(const aq_packed* w, const float* bias, void* y, int ldy);
 bool rows_supported(int M, int K);
 bool rows_fusable(int M, int K);
 cudaError_t launch_decode_rows(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
-                               const float* sx, int M, int ydtype, int32_t* P, void* ws, cudaStream_t st);
+                               const float* sx, int M, int ydtype, int32_t* P, void* ws,
+                               cudaStream_t st);
+// The streaming decode kernel (1-2 tokens; same arguments).  stream_supported: whether its shared memory fits a launch over
+// `rows` concatenated output rows.
+bool stream_supported(int M, int K, int rows);
+cudaError_t launch_decode_stream(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
+                                 const float* sx, int M, int ydtype, int32_t* P, void* ws,
+                                 cudaStream_t st);
+// The CUDA-core decode path: the streaming kernel where it applies, else the
+// register-ring kernel.  x (fused activation preparation) requires
+// cc_fusable(M, K).
+bool cc_fusable(int M, int K, int rows);
+cudaError_t launch_decode_cc(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
+                             const float* sx, int M, int ydtype, int32_t* P, void* ws,
+                             cudaStream_t st);
 
 // Split-K plan of the decode kernels (a pure function of the geometry, so
 // the workspace size and the launch agree).
@@ -88,7 +102,8 @@ cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, con
 size_t expanded_bytes(const aq_packed* w);
 cudaError_t launch_expand_int8(const aq_packed* w, void* buf, aq_packed* out, cudaStream_t st);
 cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
-                      int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st);
+                      int ydtype, int ldy, void* ws, int32_t* P, int phase,
+                      cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers
 #if defined(__CUDACC__)
@@ -315,7 +330,7 @@ __device__ __forceinline__ double act_scale(float amax) {
 __device__ __forceinline__ float act_recip(double s) { return __frcp_rn(static_cast<float>(s)); }
 
 // clamp(rint(fl64(x / s)), -127, 127): the oracle's rule, by fp64 division.
-static __device__ __noinline__ int quant_code_exact(float x, double s) {
+static __device__ __forceinline__ int quant_code_exact(float x, double s) {
   const double q = rint(static_cast<double>(x) / s);
   return static_cast<int>(fmin(fmax(q, -127.0), 127.0));
 }
@@ -342,7 +357,9 @@ __device__ __forceinline__ uint2 quantize8(const uint4& v, double s, float r32) 
   }
   if (__any_sync(__activemask(), slow)) {
     if (slow) {
-#pragma unroll 1
+      // unrolled: a runtime index would put code[] and xf[] in local memory for
+      // the fast path too
+#pragma unroll
       for (int i = 0; i < 8; ++i) code[i] = quant_code_exact(xf[i], s);
     }
   }
@@ -356,6 +373,13 @@ __device__ __forceinline__ uint2 quantize8(const uint4& v, double s, float r32) 
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
+// Start moving `bytes` (a multiple of 16, 16-byte aligned) from HBM into L2;
+// no shared memory, no completion to wait for.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
 }
 
 #endif  // __CUDACC__
@@ -381,12 +405,14 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
 // Opt a kernel in to `bytes` of dynamic shared memory on the current device.
 // The attribute is per device, so it is set once per (kernel, device); the
 // flags are atomics, so concurrent host threads at worst set it twice.
-bool set_smem_attr_once(const void* kernel, int bytes, std::atomic<bool>* done_flags);
+// carveout_pct >= 0 also sets the preferred shared-memory carveout (percent).
+bool set_smem_attr_once(const void* kernel, int bytes, int carveout_pct, std::atomic<bool>* done_flags);
 template <auto Kernel>
-cudaError_t ensure_smem_attr(int bytes) {
+cudaError_t ensure_smem_attr(int bytes, int carveout_pct = -1) {
   static std::atomic<bool> done[kMaxDevices];
-  return set_smem_attr_once(reinterpret_cast<const void*>(Kernel), bytes, done) ? cudaSuccess
-                                                                               : cudaErrorInvalidValue;
+  return set_smem_attr_once(reinterpret_cast<const void*>(Kernel), bytes, carveout_pct, done)
+             ? cudaSuccess
+             : cudaErrorInvalidValue;
 }
 
 }  // namespace aq

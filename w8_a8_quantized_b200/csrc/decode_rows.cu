@@ -63,12 +63,6 @@ struct RowsArgs {
 
 __device__ __forceinline__ int dp4a(uint32_t a, uint32_t b, int c) { return __dp4a((int)a, (int)b, c); }
 
-// Start moving `bytes` (a multiple of 16, 16-byte aligned) from HBM into L2;
-// no shared memory, no completion to wait for.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes) : "memory");
-}
-
 // Exact int -> float for |v| < 2^22 with an integer add and a float subtract.
 __device__ __forceinline__ float small_int_to_float(int v) {
   return __int_as_float(v + 0x4B400000) - 12582912.0f;

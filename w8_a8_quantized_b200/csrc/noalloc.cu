@@ -70,7 +70,7 @@ extern "C" int aq_linear_decode_noalloc(const aq_packed* w, const int8_t* xq, co
   cudaError_t e;
   if (plan.kernel == 0) {
     const DecodeProj d = decode_proj(w, bias, y, ldy);
-    e = launch_decode_rows(&d, 1, w->K, nullptr, 0, xq, sx, M, ydtype, nullptr, scratch, st);
+    e = launch_decode_cc(&d, 1, w->K, nullptr, 0, xq, sx, M, ydtype, nullptr, scratch, st);
   } else {
     e = launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, scratch, nullptr, AQ_PHASE_DECODE, st);
   }
