@@ -272,6 +272,25 @@ int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int M, int phas
                            void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Test entry for the failure path of the tensor-core linear kernel (the one that
+ * runs prefill and decode from 5 tokens): it runs that kernel with a stage that
+ * can never fill, without any invalid memory access.  The weight producer stops
+ * after `stop_after` input tiles, so the MMA issuer's wait for the next stage,
+ * and then every other role's wait, runs out; every bounded wait gives up after
+ * `wait_ns` (100 us .. 10 s) instead of the normal 2 s.  The kernel records
+ * AQ_ERR_TIMEOUT in `ws` with the code of the first wait that gave up, frees
+ * its tensor memory and returns; y (fp32 [M][ldy]) is then unspecified.
+ * aq_workspace_status() reports the error and restores the workspace (error
+ * word and split-K counters), after which the workspace serves ordinary calls.
+ * phase: AQ_PHASE_PREFILL, or AQ_PHASE_DECODE with an M that the tensor-core
+ * kernel serves.  Not a hot-path call.
+ * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ */
+int aq_debug_linear_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, int phase, float* y,
+                            int ldy, void* ws, size_t ws_bytes, unsigned long long wait_ns, int stop_after,
+                            void* stream);
+
+/*
  * Shared-input projection group (Sec. 3.3 "Shared activation preparation";
  * App. E.4): G (1..3) projections that read the same activations, e.g. query /
  * key / value or gate / up, prepared once and computed in as few launches as
@@ -324,6 +343,19 @@ size_t aq_group_workspace_bytes(int phase, int M, const aq_packed* const* w, int
  */
 int aq_linear_decode_noalloc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
                              void* y, int ydtype, int ldy, void* stream);
+
+/*
+ * Measurement helper, not part of the layer: the dense INT8 tensor-core rate of
+ * the current GPU.  One CTA per SM issues `iters` x 4 back-to-back
+ * tcgen05.mma.kind::i8 instructions (M = 128, N = 256, K = 32, INT32
+ * accumulators in tensor memory) on operands resident in shared memory; *tops
+ * (host) receives 2 M N K x instructions / elapsed seconds / 1e12 (CUDA events
+ * around one launch, after a shorter warm-up launch).  Synchronizes `stream`
+ * and allocates 4 bytes of device memory.  1 <= iters <= 2^22; about 20000
+ * runs for a few milliseconds on a B200.
+ * Errors: AQ_ERR_ARG, AQ_ERR_CUDA, AQ_ERR_TIMEOUT (the completion wait gave up).
+ */
+int aq_measure_i8_peak(int iters, double* tops, void* stream);
 
 /*
  * Synchronizes `stream`, then reads and clears the error word a kernel left in

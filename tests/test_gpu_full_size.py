@@ -15,11 +15,13 @@ from w8_a8_quantized_b200 import synth
 pytestmark = pytest.mark.gpu
 
 
-def _layer_outputs(workload: str, M: int, bN=None):
+def _layer_outputs(workload: str, M: int, bN=None, frac8=None):
     """One layer of the workload, stepped once as the benchmark does."""
     wl = dict(bench.WORKLOADS[workload])
     if bN is not None:
         wl["bN"] = bN
+    if frac8 is not None:
+        wl["frac8"] = frac8
     m = bench.Model(wl, M, torch.device("cuda"), 0, layers=1)
     m.step("group")
     torch.cuda.synchronize()
@@ -60,3 +62,30 @@ def test_dense8b_prefill_layer_full_size(bN):
 def test_qwen3_14b_prefill_chunk_full_size():
     wl, m = _layer_outputs("prefill-qwen3-14b", 8192)
     _check_sampled(wl, m, n_rows=6, n_cols=12, seed=8192)
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_single_2048_layer_as_specified(M):
+    """The single 2048 x 2048 layer: 128 x 128 tiles, 50% INT8, M = 1 and 16."""
+    wl, m = _layer_outputs("decode-single-2048", M)
+    assert (wl["bN"], wl["frac8"]) == (128, 0.5)
+    _check_sampled(wl, m, n_rows=M, n_cols=256, seed=20 + M)
+
+
+# 8B-class decode: 64- and 128-row tiles across the INT8 fractions and token
+# counts (1: streaming CUDA-core kernel; 5: tensor cores, two 64-row tile rows
+# per 128-row accumulator block; 16 and 64: tensor cores with split reduction)
+@pytest.mark.parametrize("bN,frac8,M", [(64, 0.0, 1), (64, 0.25, 5), (64, 0.5, 16), (64, 1.0, 64),
+                                        (64, 0.5, 1), (64, 0.25, 64), (128, 0.5, 1), (128, 1.0, 16)])
+def test_dense8b_decode_layer_full_size(bN, frac8, M):
+    wl, m = _layer_outputs("decode-dense-8b", M, bN=bN, frac8=frac8)
+    _check_sampled(wl, m, n_rows=M, n_cols=48, seed=30 + M)
+
+
+@pytest.mark.parametrize("M", [1, 2, 16, 64])
+def test_qwen3_14b_decode_layer_full_size(M):
+    """K = 17408 in the MLP down projection: at 2 tokens its activations do not
+    fit the fused preparation, so it runs as activation quantization plus the
+    CUDA-core kernel on the codes."""
+    wl, m = _layer_outputs("decode-qwen3-14b", M)
+    _check_sampled(wl, m, n_rows=M, n_cols=32, seed=40 + M)

@@ -24,7 +24,8 @@ EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "
             "aq_workspace_bytes", "aq_linear_decode", "aq_linear_prefill", "aq_debug_tile_partials",
             "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc",
             "aq_quantize_weights", "aq_paper_packed_bytes", "aq_expanded_bytes", "aq_expand_int8",
-            "aq_linear_prefill_expanded", "aq_act_group_rows", "aq_quant_act_groups")
+            "aq_linear_prefill_expanded", "aq_act_group_rows", "aq_quant_act_groups", "aq_measure_i8_peak",
+            "aq_debug_linear_stalled")
 
 
 class AqError(RuntimeError):
@@ -95,6 +96,11 @@ def lib():
     L.aq_group_workspace_bytes.argtypes = [c_int, c_int, ctypes.POINTER(P), c_int]
     L.aq_linear_decode_noalloc.restype = c_int
     L.aq_linear_decode_noalloc.argtypes = [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_void_p]
+    L.aq_debug_linear_stalled.restype = c_int
+    L.aq_debug_linear_stalled.argtypes = [P, c_void_p, c_void_p, c_int, c_int, c_void_p, c_int, c_void_p, c_size_t,
+                                          ctypes.c_ulonglong, c_int, c_void_p]
+    L.aq_measure_i8_peak.restype = c_int
+    L.aq_measure_i8_peak.argtypes = [c_int, ctypes.POINTER(ctypes.c_double), c_void_p]
     L.aq_workspace_status.restype = c_int
     L.aq_workspace_status.argtypes = [c_void_p, c_void_p, ctypes.POINTER(c_int)]
     _lib = L
@@ -467,6 +473,18 @@ def aq_debug_tile_partials(w: PackedWeights, xq: torch.Tensor, phase: int, ws=No
     return P
 
 
+def aq_debug_linear_stalled(w: PackedWeights, xq, sx, phase: int, ws: torch.Tensor, wait_ns: int = 20_000_000,
+                            stop_after: int = 1) -> torch.Tensor:
+    """Run the tensor-core linear kernel with a stage that never fills (test of the
+    bounded waits): returns the (unspecified) output; the error lands in `ws`."""
+    M, out = _linear_operands(w, xq, sx, None, None, torch.float32)
+    with torch.cuda.device(w.device):
+        _check(lib().aq_debug_linear_stalled(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M, phase,
+                                             out.data_ptr(), out.stride(0), ws.data_ptr(), ws.numel(), wait_ns,
+                                             stop_after, _stream(w.device)), "aq_debug_linear_stalled")
+    return out
+
+
 def aq_workspace_status(ws: torch.Tensor):
     """Synchronise; return (status, info) of the kernel error word of a workspace and clear it."""
     info = ctypes.c_int(0)
@@ -474,6 +492,16 @@ def aq_workspace_status(ws: torch.Tensor):
     if rc not in (AQ_OK, -7):
         _check(rc, "aq_workspace_status")
     return rc, info.value
+
+
+def aq_measure_i8_peak(iters: int = 20000, device=None) -> float:
+    """Measured dense INT8 tensor-core rate of the device in TOPS (tcgen05 loop on
+    shared-memory operands; a measurement helper, not part of the layer)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    tops = ctypes.c_double(0.0)
+    with torch.cuda.device(dev):
+        _check(lib().aq_measure_i8_peak(iters, ctypes.byref(tops), _stream(dev)), "aq_measure_i8_peak")
+    return float(tops.value)
 
 
 def check_all_workspaces():

@@ -267,6 +267,22 @@ extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int 
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
 }
 
+extern "C" int aq_debug_linear_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, int phase,
+                                       float* y, int ldy, void* ws, size_t ws_bytes, unsigned long long wait_ns,
+                                       int stop_after, void* stream) {
+  int rc = check_linear(w, xq, sx, M, y, AQ_F32, ldy);
+  if (rc != AQ_OK) return rc;
+  if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return AQ_ERR_ARG;
+  if (phase == AQ_PHASE_DECODE && (M > kMaxDecodeM || plan_decode(M, w).kernel != 1)) return AQ_ERR_ARG;
+  if (wait_ns < 100000ull || wait_ns > 10000000000ull || stop_after < 0) return AQ_ERR_ARG;
+  const size_t need = phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w) : prefill_ws_bytes(M, w);
+  if (!ws || ws_bytes < need) return AQ_ERR_WORKSPACE;
+  return launch_tc_stalled(w, xq, sx, M, y, ldy, ws, phase, wait_ns, stop_after, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? AQ_OK
+             : AQ_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- shared-input groups (App. E.4)
 static int check_group(int phase, const aq_packed* const* w, int G, const uint16_t* x, int ldx, int M) {
   if (!w || G < 1 || G > kMaxGroup || !x || M < 1) return AQ_ERR_ARG;

@@ -79,8 +79,7 @@ cudaError_t launch_decode_stream(const DecodeProj* projs, int G, int K, const ui
 // cc_fusable(M, K).
 bool cc_fusable(int M, int K, int rows);
 cudaError_t launch_decode_cc(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
-                             const float* sx, int M, int ydtype, int32_t* P, void* ws,
-                             cudaStream_t st);
+                             const float* sx, int M, int ydtype, int32_t* P, void* ws, cudaStream_t st);
 
 // Split-K plan of the decode kernels (a pure function of the geometry, so
 // the workspace size and the launch agree).
@@ -102,8 +101,11 @@ cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, con
 size_t expanded_bytes(const aq_packed* w);
 cudaError_t launch_expand_int8(const aq_packed* w, void* buf, aq_packed* out, cudaStream_t st);
 cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
-                      int ydtype, int ldy, void* ws, int32_t* P, int phase,
-                      cudaStream_t st);
+                      int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st);
+// Test form of launch_tc: every bounded wait gives up after wait_ns and the
+// weight producer stops after `stop_after` tiles (so later stages never fill).
+cudaError_t launch_tc_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, void* y, int ldy,
+                              void* ws, int phase, unsigned long long wait_ns, int stop_after, cudaStream_t st);
 
 // ---------------------------------------------------------------- device helpers
 #if defined(__CUDACC__)
@@ -164,16 +166,17 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 }
 
 // Wait for the phase with the given parity to complete.  Returns false when
-// `abort` became nonzero or the time limit passed; never waits unbounded.
+// `abort` became nonzero or `limit_ns` passed; never waits unbounded.
 // Between checks of the abort flag and the clock the thread sleeps (see
 // mbar_try_wait_sleep), so the checks cost little.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -138,6 +138,8 @@ struct TcArgs {
   float* partial;  // [S][N][Mp], Mp = M rounded up to a multiple of 4
   int* counters;   // [nrb * ntb]
   int ws_clear;    // bytes of split-K counters after the workspace header (0 without splits)
+  unsigned long long wait_ns;  // limit of every bounded wait (kWaitTimeoutNs; shorter in the stall test)
+  int stop_after;  // >= 0: the weight producer stops after this many tiles (stall test); -1 otherwise
   int32_t* P;      // debug: exact tile products [M][N][C], or null
 };
 
@@ -394,11 +396,15 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       RingPos mr{0, 0}, sr{0, 0};
       bool ok = true;
       for (uint32_t g = 0; g < g_total; ++g) {
-        if (!mbar_wait(&meta_full[mr.i], mr.ph, abort_flag)) { fail(1); ok = false; break; }
+        if (a.stop_after >= 0 && g >= (uint32_t)a.stop_after) {  // stall test: later stages never fill
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&meta_full[mr.i], mr.ph, abort_flag, a.wait_ns)) { fail(1); ok = false; break; }
         const MetaRec rec = meta[mr.i];
         mbar_arrive(&meta_empty[mr.i]);
         mr.next<kMetaSlots>();
-        if (g >= (uint32_t)S_ && !mbar_wait(&mma_done[(g - S_) % kDone], ((g - S_) / kDone) & 1, abort_flag)) {
+        if (g >= (uint32_t)S_ && !mbar_wait(&mma_done[(g - S_) % kDone], ((g - S_) / kDone) & 1, abort_flag, a.wait_ns)) {
           fail(2);
           ok = false;
           break;
@@ -419,7 +425,12 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         }
         sr.next<S_>();
       }
-      if (!ok || *abort_flag) abort_grace();
+      if (!ok || *abort_flag) {
+        // (stall test: wait for the other roles to give up, then for copies in flight)
+        const unsigned long long t0 = globaltimer_ns();
+        while (!*abort_flag && globaltimer_ns() - t0 < 2 * a.wait_ns) __nanosleep(1000);
+        abort_grace();
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -430,10 +441,10 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       RingPos sr{0, 0}, br{0, 0};
       uint32_t g = 0;
       for (; g < g_total; ++g) {
-        if (!mbar_wait(&full[sr.i], sr.ph, abort_flag)) { fail(4); break; }
-        if (!mbar_wait(&expanded[sr.i], sr.ph, abort_flag)) { fail(5); break; }
+        if (!mbar_wait(&full[sr.i], sr.ph, abort_flag, a.wait_ns)) { fail(4); break; }
+        if (!mbar_wait(&expanded[sr.i], sr.ph, abort_flag, a.wait_ns)) { fail(5); break; }
         // use u of a buffer waits for the epilogue's release number u (release 0 = initial bias)
-        if (!mbar_wait(&tmem_empty[br.i], br.ph, abort_flag)) { fail(6); break; }
+        if (!mbar_wait(&tmem_empty[br.i], br.ph, abort_flag, a.wait_ns)) { fail(6); break; }
         tc_fence_after();
         const uint64_t soff = (uint64_t)((sr.i * Sh::kStageBytes) >> 4);  // descriptor address field: 16-byte units
         const uint32_t d = tmem_base + br.i * NT;
@@ -447,7 +458,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       }
       if (g > 0) {  // every MMA issued is complete before tensor memory is freed
         mma_commit(drain);
-        mbar_wait(drain, 0, never_flag);
+        mbar_wait(drain, 0, never_flag, a.wait_ns);
       }
     }
   } else if (warp == 2) {
@@ -467,7 +478,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       if (u >= a.units) break;
       const int j = x.j0 + (int)(g - base);
       const int ms = g % kMetaSlots;
-      if (!mbar_wait(&meta_empty[ms], ((g / kMetaSlots) & 1) ^ 1, abort_flag)) { fail(7); break; }
+      if (!mbar_wait(&meta_empty[ms], ((g / kMetaSlots) & 1) ^ 1, abort_flag, a.wait_ns)) { fail(7); break; }
       uint32_t kinds = 0, bytes8 = 0, bytes4 = 0, row[2] = {0, 0};
       for (int sub = 0; sub < a.tpb; ++sub) {
         const int r = x.rb * a.tpb + sub;
@@ -498,7 +509,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       RingPos sr{0, 0};
       bool ok = true;
       for (uint32_t g = 0; g < g_total; ++g, bi.next(a)) {
-        if (g >= (uint32_t)S_ && !mbar_wait(&mma_done[(g - S_) % kDone], ((g - S_) / kDone) & 1, abort_flag)) {
+        if (g >= (uint32_t)S_ && !mbar_wait(&mma_done[(g - S_) % kDone], ((g - S_) / kDone) & 1, abort_flag, a.wait_ns)) {
           fail(3);
           ok = false;
           break;
@@ -523,7 +534,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
     RingPos sr{0, 0};
     for (uint32_t g = 0; g < g_total; ++g) {
       const int st = sr.i;
-      if (!__all_sync(0xffffffffu, mbar_wait(&staged[st], sr.ph, abort_flag))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&staged[st], sr.ph, abort_flag, a.wait_ns))) {
         fail(8);
         break;
       }
@@ -608,8 +619,8 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         const uint32_t gl = g + nt - 1;
         // the scale slot of the pair's last tile implies the first one's (the
         // transform warps arrive in tile order)
-        if (!__all_sync(0xffffffffu, mbar_wait(&mma_done[gl % kDone], (gl / kDone) & 1, abort_flag) &&
-                                         mbar_wait(&sw_full[gl % kSwRing], (gl / kSwRing) & 1, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&mma_done[gl % kDone], (gl / kDone) & 1, abort_flag, a.wait_ns) &&
+                                         mbar_wait(&sw_full[gl % kSwRing], (gl / kSwRing) & 1, abort_flag, a.wait_ns))) {
           fail(9);
           ok = false;
           break;
@@ -722,11 +733,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       }
       __threadfence();
       mbar_arrive(epi_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag))) { fail(11); ok = false; continue; }
+      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag, a.wait_ns))) { fail(11); ok = false; continue; }
       sync_phase ^= 1;
       if (ew == 0 && lane == 0) *last_flag = (atomicAdd(a.counters + x.rb * a.ntb + x.tb, 1) == a.S - 1);
       mbar_arrive(epi_sync);
-      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag))) { fail(12); ok = false; continue; }
+      if (!__all_sync(0xffffffffu, mbar_wait(epi_sync, sync_phase, abort_flag, a.wait_ns))) { fail(12); ok = false; continue; }
       sync_phase ^= 1;
       if (*last_flag) {
         __threadfence();
@@ -802,9 +813,12 @@ cudaError_t launch_nt(const aq_packed* w, const int8_t* xq, TcArgs a, int grid, 
 
 }  // namespace
 
-cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
-                      int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st) {
+static cudaError_t launch_tc_impl(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                                  void* y, int ydtype, int ldy, void* ws, int32_t* P, int phase,
+                                  unsigned long long wait_ns, int stop_after, cudaStream_t st) {
   TcArgs a;
+  a.wait_ns = wait_ns;
+  a.stop_after = stop_after;
   a.bitmap = w->bitmap; a.tile_idx = w->tile_idx; a.scales = w->scales;
   a.N = w->N; a.K = w->K; a.bN = w->bN; a.R = w->R; a.C = w->C; a.T4 = w->T4; a.T8 = w->T8;
   a.tpb = 128 / w->bN;
@@ -867,6 +881,16 @@ cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int
 #undef AQ_TC_CASE_WIDE
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
+                      int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st) {
+  return launch_tc_impl(w, xq, sx, M, bias, y, ydtype, ldy, ws, P, phase, kWaitTimeoutNs, -1, st);
+}
+
+cudaError_t launch_tc_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, void* y, int ldy,
+                              void* ws, int phase, unsigned long long wait_ns, int stop_after, cudaStream_t st) {
+  return launch_tc_impl(w, xq, sx, M, nullptr, y, AQ_F32, ldy, ws, nullptr, phase, wait_ns, stop_after, st);
 }
 
 }  // namespace aq
