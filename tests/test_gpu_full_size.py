@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 def _layer_outputs(workload: str, M: int, bN=None, frac8=None):
     """One layer of the workload, stepped once as the benchmark does."""
-    wl = dict(bench.WORKLOADS[workload])
+    wl = dict(bench.WORKLOADS[workload], gen="host")  # the oracle regenerates the host-drawn values
     if bN is not None:
         wl["bN"] = bN
     if frac8 is not None:

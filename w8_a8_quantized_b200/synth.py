@@ -32,7 +32,7 @@ import numpy as np
 __all__ = [
     "MODELS", "projections", "precision_map", "weight_codes", "weight_scales",
     "activations", "f32_to_bf16_bits", "projection_inputs", "SingleProjection",
-    "float_weights",
+    "float_weights", "device_projection_inputs", "device_activations",
 ]
 
 # (hidden, q-proj out, k/v-proj out, MLP intermediate, layers)
@@ -149,3 +149,44 @@ def projection_inputs(N: int, K: int, bN: int, bK: int, frac_int8: float, seed) 
     return SingleProjection(N, K, bN, bK, pmap,
                             weight_codes(N, K, pmap, bN, bK, seed),
                             weight_scales(N, C, seed))
+
+
+def device_projection_inputs(N: int, K: int, bN: int, bK: int, frac_int8: float, seed, device):
+    """The recipe of projection_inputs drawn with torch's generator on a CUDA
+    device (for models too large to draw on the host in reasonable time): map
+    with exactly round_half_even(f*R*C) INT8 tiles chosen by a seeded
+    permutation, codes uniform over [-128, 127] in INT8 tiles and [-8, 7] in INT4
+    tiles, scales uniform in [1e-3, 1e-2] rounded to fp16.  The same seed gives
+    the same values on any device of the same kind; they differ from
+    projection_inputs' values (another generator).  Returns (codes int8 [N][K],
+    scales float16 [N][C], pmap uint8 [R][C]) on `device`."""
+    import torch
+    R, C = N // bN, K // bK
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence(list(_key(seed))).generate_state(1, np.uint64)[0] >> 1))
+    T = R * C
+    t8 = int(round(frac_int8 * T))
+    pmap = torch.ones(T, dtype=torch.uint8, device=device)
+    pmap[torch.randperm(T, generator=g, device=device)[:t8]] = 0
+    pmap = pmap.view(R, C)
+    raw = torch.randint(-128, 128, (N, K), dtype=torch.int16, generator=g, device=device)
+    int4 = pmap.bool().repeat_interleave(bN, 0).repeat_interleave(bK, 1)
+    codes = torch.where(int4, (raw & 15) - 8, raw).to(torch.int8)
+    scales = (torch.rand((N, C), dtype=torch.float32, generator=g, device=device) * 9e-3 + 1e-3).to(torch.float16)
+    return codes, scales, pmap
+
+
+def device_activations(M: int, K: int, seed, device, outlier_frac: float = 0.0, outlier_mult: float = 20.0):
+    """The recipe of activations drawn with torch's generator on a CUDA device:
+    bf16 [M][K] N(0,1) values, round(outlier_frac*K) seeded input channels
+    multiplied by outlier_mult.  Other values than activations' (another
+    generator)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence(list(_key(seed)) + [4]).generate_state(1, np.uint64)[0] >> 1))
+    x = torch.randn((M, K), dtype=torch.float32, generator=g, device=device)
+    n_out = int(round(outlier_frac * K))
+    if n_out:
+        cols = torch.randperm(K, generator=g, device=device)[:n_out]
+        x[:, cols] *= outlier_mult
+    return x.to(torch.bfloat16)
