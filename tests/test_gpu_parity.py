@@ -221,6 +221,33 @@ def test_decode_long_rows_reuse_every_ring_slot(M, N, K, bN):
 
 
 @pytest.mark.parametrize("M", [1, 2])
+@pytest.mark.parametrize("N,K,bN", [(4096, 8192, 128), (2560, 14336, 64)])
+def test_decode_wide_launch(M, N, K, bN):
+    """Launches above 200 K weights per SM: at 1 token the streaming kernel takes
+    its wide shape (16 warps, 3-stage rings, one CTA per SM).  Outputs against
+    the oracle, per-tile products bit-exact."""
+    p, x, w, xq, sx = packed_case(N, K, bN, 0.4, 1600 + M + N, M, outlier=0.01)
+    assert_output_close(aq.aq_linear_decode(w, xq, sx), oracle_linear(p, x))
+    P = aq.aq_debug_tile_partials(w, xq, aq.AQ_PHASE_DECODE)
+    assert np.array_equal(P.cpu().numpy(), oracle.tile_partials(p.codes, oracle.quant_act(x)[0], 128))
+
+
+def test_group_fused_wide_launch():
+    """A gate/up-style group of 2 x 8192 rows over K = 4096 at 1 token: one fused
+    launch (activation preparation inside) in the wide shape."""
+    shapes = [(8192, 4096), (8192, 4096)]
+    ps, ws, x = _group_case(shapes, 1, 1700, aq.AQ_PHASE_DECODE)
+    grp = aq.Group(ws, aq.AQ_PHASE_DECODE, 1)
+    outs = [torch.empty((1, N), device="cuda") for N, _ in shapes]
+    for _ in range(2):
+        grp(dev_bf16(x), outs)
+    for p, o in zip(ps, outs):
+        assert_output_close(o, oracle_linear(p, x))
+    rc, _ = aq.aq_workspace_status(grp.ws)
+    assert rc == 0
+
+
+@pytest.mark.parametrize("M", [1, 2])
 def test_group_fused_long_rows(M):
     """A fused q/k/v-style group whose CTAs each stream several row blocks of 40
     tile columns (ring slots refilled many times)."""

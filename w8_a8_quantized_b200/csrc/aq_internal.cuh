@@ -303,14 +303,16 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
 // ---- per-token INT8 activation quantization (shared by every kernel that prepares activations)
+// max(m, |x|) over eight bf16 values.  |x| of a bf16 is its bit pattern with the
+// sign cleared, and for non-negative values the float order is the integer order
+// of the patterns, so the eight magnitudes reduce with 16-bit-pair integer maxima
+// and one conversion at the end.  (A NaN pattern converts to NaN, which fmaxf
+// ignores.)
 __device__ __forceinline__ float abs_max8(const uint4& v, float m) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = fmaxf(m, bf16_bits_to_float(w[i] & 0x7FFFu));
-    m = fmaxf(m, bf16_bits_to_float((w[i] >> 16) & 0x7FFFu));
-  }
-  return m;
+  const uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  const uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+  const uint32_t c = __vmaxu2(a, b);
+  return fmaxf(m, bf16_bits_to_float(max(c & 0xFFFFu, c >> 16)));
 }
 
 // s = max(fl64(amax / 127), 1e-12) (eq. 6 floor).  The quotient is formed from
@@ -341,37 +343,43 @@ static __device__ __forceinline__ int quant_code_exact(float x, double s) {
 // Eight codes of clamp(rint(fl64(x / s)), -127, 127).
 // Fast path: t = x * r32 carries at most three roundings of 2^-24 each
 // (fp32(s), the reciprocal, the product), so |t - x/s| <= 127 * 3 * 2^-24
-// < 2.3e-5 (|x / s| <= 127).  When t is more than 4e-5 away from the nearest
-// half-integer the exact quotient, and its fp64 rounding, round to the same
-// integer as t.  Ties and near-ties (rare) are redone by fp64 division; the
-// warp votes so that the division is a real branch, never paid by every element.
+// < 2.3e-5 (|x / s| <= 127).  The rounding is done on the FMA pipe: for
+// |c| < 2^22, c + 1.5 * 2^23 holds rint(c) (ties to even) in its low mantissa
+// bits, so with c = clamp(t, -127, 127) the low byte of that sum's pattern is the
+// two's-complement code and subtracting 1.5 * 2^23 again gives k = rint(c)
+// exactly (clamping before rounding equals clamping after it for integer
+// bounds).  When t is more than 4e-5 away from the nearest half-integer, the
+// exact quotient rounds, and clamps, to the same code (for t > 127.49996 the
+// test below fails and the element takes the exact path).  Ties and near-ties
+// (rare) are redone by fp64 division; the warp votes so that the division is a
+// real branch, never paid by every element.
 __device__ __forceinline__ uint2 quantize8(const uint4& v, double s, float r32) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   float xf[8];
-  int code[8];
+  uint32_t u[8];
   bool slow = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     xf[i] = bf16_bits_to_float((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
     const float t = xf[i] * r32;
-    const float k = rintf(t);
+    const float r = __fadd_rn(fminf(fmaxf(t, -127.f), 127.f), kRound);
+    const float k = __fsub_rn(r, kRound);
     slow |= !(0.5f - fabsf(t - k) > 4.0e-5f);
-    code[i] = static_cast<int>(fminf(fmaxf(k, -127.f), 127.f));
+    u[i] = __float_as_uint(r);
   }
   if (__any_sync(__activemask(), slow)) {
     if (slow) {
-      // unrolled: a runtime index would put code[] and xf[] in local memory for
+      // unrolled: a runtime index would put u[] and xf[] in local memory for
       // the fast path too
 #pragma unroll
-      for (int i = 0; i < 8; ++i) code[i] = quant_code_exact(xf[i], s);
+      for (int i = 0; i < 8; ++i) u[i] = static_cast<uint32_t>(quant_code_exact(xf[i], s));
     }
   }
-  uint32_t out[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-    out[h] = (uint32_t)(code[4 * h] & 0xFF) | ((uint32_t)(code[4 * h + 1] & 0xFF) << 8) |
-             ((uint32_t)(code[4 * h + 2] & 0xFF) << 16) | ((uint32_t)(code[4 * h + 3] & 0xFF) << 24);
-  return make_uint2(out[0], out[1]);
+  // low bytes of u[0..3] and u[4..7]
+  const uint32_t l0 = __byte_perm(u[0], u[1], 0x0040), h0 = __byte_perm(u[2], u[3], 0x0040);
+  const uint32_t l1 = __byte_perm(u[4], u[5], 0x0040), h1 = __byte_perm(u[6], u[7], 0x0040);
+  return make_uint2(__byte_perm(l0, h0, 0x5410), __byte_perm(l1, h1, 0x5410));
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {

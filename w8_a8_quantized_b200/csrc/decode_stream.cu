@@ -15,9 +15,16 @@
 // kernel.  So every warp starts copying its first stages of weights into
 // shared memory as soon as its CTA is resident, before the wait, and only the
 // activation preparation, the products and the reduction follow the wait.  The
-// grid has one CTA per SM and a CTA keeps its shared memory near 104 KB, so the
-// CTAs of two consecutive launches fit on every SM side by side: while one
-// launch computes, the next one already streams its weights.  (A register-ring
+// grid has one CTA per SM.  For launches of up to 100 K weights per SM a CTA
+// keeps its shared memory near 104 KB, so the CTAs of two consecutive launches
+// fit on every SM side by side: while one launch computes, the next one already
+// streams its weights.  Larger launches take the wide shape: one CTA of 16 warps
+// with 3-stage rings fills the SM and keeps more bytes in flight through the
+// long stream, at the price of the next launch starting its copies only when
+// this CTA leaves.  (Measured at 1 token: 8B-class layers 17-20% faster than
+// with the narrow shape alone, 14B-class layers 1.6x; a threshold of 200 K made
+// the 3B-class model 15% slower, every change of shape between consecutive
+// launches costing the next launch its early start.)  (A register-ring
 // design that issued its loads from every thread measured a launch-long
 // dependent chain: its loads could only start once a CTA had a slot, and a CTA
 // only got a slot when the previous launch left.)
@@ -60,16 +67,27 @@
 namespace aq {
 namespace {
 
-constexpr int kWarps = 12;  // 2 per SM sub-partition left the stage loop latency-bound
-constexpr int kStreamThreads = 32 * kWarps;
-constexpr int kRing = 2;                         // stages in flight per warp
 constexpr int kMaxR = 32;                        // rows of a row block (stage), at most
 constexpr int kSlotBytes = kMaxR * kTileK;       // one stage: up to 32 rows of an INT8 tile
 constexpr int kSlotScBytes = kMaxR * 2;          // the stage's fp16 row scales
 constexpr int kMaxBlocks = 16;
 constexpr int kMaxCtaRows = 256;
-constexpr size_t kRingBytes = (size_t)kWarps * kRing * (kSlotBytes + kSlotScBytes);
-constexpr size_t kSmemLimit = 112 * 1024;        // per CTA: two launches' CTAs on one SM (228 KB)
+
+// The two shapes of the kernel: warps per CTA, stages in flight per warp, CTAs per
+// SM the shape is built for, and its shared-memory limit per CTA.
+template <int WARPS, int RING, int CTAS_PER_SM, int SMEM_KB>
+struct StreamShape {
+  static constexpr int kWarps = WARPS, kRing = RING, kCtasPerSm = CTAS_PER_SM;
+  static constexpr int kThreads = 32 * WARPS;
+  static constexpr size_t kRingBytes = (size_t)WARPS * RING * (kSlotBytes + kSlotScBytes);
+  static constexpr size_t kSmemLimit = (size_t)SMEM_KB * 1024;
+};
+// 12 warps (fewer left the stage loop latency-bound), 2 stages each: two launches' CTAs per SM (228 KB)
+using ShapeShared = StreamShape<12, 2, 2, 112>;
+// 16 warps, 3 stages each: one CTA per SM (220 KB dynamic + static shared memory < 227 KB)
+using ShapeWide = StreamShape<16, 3, 1, 220>;
+// launches with more weights than this per SM take the wide shape
+constexpr long long kWideWeightsPerSm = 100 * 1024;
 
 struct SProj {
   const uint8_t* bitmap;
@@ -148,8 +166,10 @@ struct StageRec {
 };
 
 // (two CTAs per SM: the running launch and the next one, which streams its weights)
-template <int MT, bool FUSED, bool DEBUG>
-__global__ void __launch_bounds__(kStreamThreads, 2) decode_stream_kernel(const __grid_constant__ SArgs a) {
+template <class Shape, int MT, bool FUSED, bool DEBUG>
+__global__ void __launch_bounds__(Shape::kThreads, Shape::kCtasPerSm) decode_stream_kernel(const __grid_constant__ SArgs a) {
+  constexpr int kWarps = Shape::kWarps, kRing = Shape::kRing, kStreamThreads = Shape::kThreads;
+  constexpr size_t kRingBytes = Shape::kRingBytes;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Block blocks[kMaxBlocks];
   __shared__ float redq[kWarps][MT];
@@ -164,15 +184,15 @@ __global__ void __launch_bounds__(kStreamThreads, 2) decode_stream_kernel(const 
   int8_t* act = reinterpret_cast<int8_t*>(smem + kRingBytes);  // [MT][K] codes
   float* red = reinterpret_cast<float*>(act + (size_t)MT * K);  // [kWarps][cta_rows][MT]
 
-  const int lo = (int)((long long)a.strips * blockIdx.x / gridDim.x) * 8;
-  const int hi = (int)((long long)a.strips * (blockIdx.x + 1) / gridDim.x) * 8;
+  const int lo = (int)((unsigned)a.strips * blockIdx.x / gridDim.x) * 8;  // (strips x grid < 2^32)
+  const int hi = (int)((unsigned)a.strips * (blockIdx.x + 1) / gridDim.x) * 8;
   if (threadIdx.x == 0) nblocks_s = cta_blocks(a, lo, hi, blocks);
   __syncthreads();
   const int nb = nblocks_s;
   if (nb < 0) return;  // the host never builds such a launch (rows per CTA are capped)
   const int T = nb * C;  // stages of the CTA: stage g is tile column g % C of row block g / C
-  const int g0 = (int)((long long)T * warp / kWarps);
-  const int Tw = (int)((long long)T * (warp + 1) / kWarps) - g0;  // this warp's stages g0 .. g0 + Tw - 1
+  const int g0 = T * warp / kWarps;
+  const int Tw = T * (warp + 1) / kWarps - g0;  // this warp's stages g0 .. g0 + Tw - 1
 
   // record of this warp's stage k (k in [32 q, 32 q + 32) for the batch q held by the lane)
   auto make_rec = [&](int k) {
@@ -443,17 +463,30 @@ __global__ void __launch_bounds__(kStreamThreads, 2) decode_stream_kernel(const 
   }
 }
 
+template <class Shape>
 size_t stream_smem(int MT, int K, int cta_rows) {
-  return kRingBytes + (size_t)MT * K + (size_t)kWarps * cta_rows * MT * 4;
+  return Shape::kRingBytes + (size_t)MT * K + (size_t)Shape::kWarps * cta_rows * MT * 4;
 }
 
-template <int MT, bool FUSED, bool DEBUG>
+template <class Shape, int MT, bool FUSED, bool DEBUG>
 cudaError_t launch_stream_t(const SArgs& a, int grid, size_t smem, cudaStream_t st) {
-  // all of the SM's unified L1 / shared storage as shared memory, so the CTAs of
-  // two consecutive launches fit side by side
-  cudaError_t e = ensure_smem_attr<decode_stream_kernel<MT, FUSED, DEBUG>>((int)kSmemLimit, 100);
+  // all of the SM's unified L1 / shared storage as shared memory (the shared shape:
+  // so that the CTAs of two consecutive launches fit side by side)
+  cudaError_t e = ensure_smem_attr<decode_stream_kernel<Shape, MT, FUSED, DEBUG>>((int)Shape::kSmemLimit, 100);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_stream_kernel<MT, FUSED, DEBUG>, dim3(grid), dim3(kStreamThreads), smem, st, a);
+  return launch_pdl(decode_stream_kernel<Shape, MT, FUSED, DEBUG>, dim3(grid), dim3(Shape::kThreads), smem, st, a);
+}
+
+template <class Shape>
+cudaError_t launch_stream_s(const SArgs& a, int grid, cudaStream_t st) {
+  const size_t smem = stream_smem<Shape>(a.M, a.K, a.cta_rows);
+  if (a.M > 2 || smem > Shape::kSmemLimit) return cudaErrorInvalidValue;
+  if (a.P != nullptr) return a.M == 1 ? launch_stream_t<Shape, 1, false, true>(a, grid, smem, st)
+                                      : launch_stream_t<Shape, 2, false, true>(a, grid, smem, st);
+  if (a.x != nullptr) return a.M == 1 ? launch_stream_t<Shape, 1, true, false>(a, grid, smem, st)
+                                      : launch_stream_t<Shape, 2, true, false>(a, grid, smem, st);
+  return a.M == 1 ? launch_stream_t<Shape, 1, false, false>(a, grid, smem, st)
+                  : launch_stream_t<Shape, 2, false, false>(a, grid, smem, st);
 }
 
 }  // namespace
@@ -467,11 +500,21 @@ static void stream_grid(int rows, int* grid, int* cta_rows) {
   *cta_rows = ((strips + *grid - 1) / *grid) * 8;
 }
 
+// The wide shape for launches above kWideWeightsPerSm weights per SM, or whose
+// activations and reduction buffer do not fit the shared shape.
+static bool stream_wide(int M, int K, int rows) {
+  int grid, cta_rows;
+  stream_grid(rows, &grid, &cta_rows);
+  return (long long)rows * K > kWideWeightsPerSm * grid ||
+         stream_smem<ShapeShared>(M, K, cta_rows) > ShapeShared::kSmemLimit;
+}
+
 bool stream_supported(int M, int K, int rows) {
   if (M < 1 || M > 2 || rows < 8) return false;
   int grid, cta_rows;
   stream_grid(rows, &grid, &cta_rows);
-  return stream_smem(M, K, cta_rows) <= kSmemLimit;
+  return stream_wide(M, K, rows) ? stream_smem<ShapeWide>(M, K, cta_rows) <= ShapeWide::kSmemLimit
+                                 : stream_smem<ShapeShared>(M, K, cta_rows) <= ShapeShared::kSmemLimit;
 }
 
 cudaError_t launch_decode_stream(const DecodeProj* projs, int G, int K, const uint16_t* x, int ldx, const int8_t* xq,
@@ -498,13 +541,8 @@ cudaError_t launch_decode_stream(const DecodeProj* projs, int G, int K, const ui
   a.strips = rows / 8;
   int grid;
   stream_grid(rows, &grid, &a.cta_rows);
-  const size_t smem = stream_smem(M, K, a.cta_rows);
-  if (M > 2 || smem > kSmemLimit) return cudaErrorInvalidValue;
-  if (P != nullptr) return M == 1 ? launch_stream_t<1, false, true>(a, grid, smem, st)
-                                  : launch_stream_t<2, false, true>(a, grid, smem, st);
-  if (x != nullptr) return M == 1 ? launch_stream_t<1, true, false>(a, grid, smem, st)
-                                  : launch_stream_t<2, true, false>(a, grid, smem, st);
-  return M == 1 ? launch_stream_t<1, false, false>(a, grid, smem, st) : launch_stream_t<2, false, false>(a, grid, smem, st);
+  if (M < 1 || M > 2) return cudaErrorInvalidValue;
+  return stream_wide(M, K, rows) ? launch_stream_s<ShapeWide>(a, grid, st) : launch_stream_s<ShapeShared>(a, grid, st);
 }
 
 }  // namespace aq
