@@ -25,7 +25,8 @@
  *    returns AQ_ERR_CUDA.  Errors found by a kernel while it runs (a bounded
  *    wait that gave up) are recorded in the workspace and reported by
  *    aq_workspace_status().
- *  - Geometry: bN in {64, 128}, bK == 128, N % bN == 0, K % bK == 0.
+ *  - Geometry: bN in {64, 128}, bK == 128, N % bN == 0, K % bK == 0.  The
+ *    paper-exact mode (aq_pack_tiles, aq_paper_*) takes bK == 64 instead.
  *  - Row-major everywhere; leading dimensions are in elements.
  */
 #ifndef AQ_H_
@@ -70,12 +71,21 @@ typedef enum { AQ_PHASE_DECODE = 0, AQ_PHASE_PREFILL = 1 } aq_phase;
  *  w8       int8   [T8][bN][bK]    INT8 tiles in row order, row-major in the tile
  *  scales   fp16   [R][C][bN]      sw[n][j] at (r*C + j)*bN + (n - r*bN), bits
  *                                  as uint16, logical tile order
+ *           (scale_kind == AQ_SCALES_TILE_FP32: fp32 [R][C], one scale per tile
+ *                                  at r*C + j, in the first 4*R*C bytes of the
+ *                                  same buffer; written by aq_pack_tiles)
+ *  scale_kind                      AQ_SCALES_ROW_FP16 (aq_pack; the per-token
+ *                                  layer's kernels take only this kind) or
+ *                                  AQ_SCALES_TILE_FP32 (aq_pack_tiles; the
+ *                                  paper-exact aq_paper_linear takes only this)
  *
  * Inside a tile both precisions use the same element order: output row, then
  * input column.  w4, w8 and scales must start on a 16-byte boundary (the
  * kernels move them with bulk copies); a packed layout that breaks this is
  * rejected with AQ_ERR_ARG.
  */
+typedef enum { AQ_SCALES_ROW_FP16 = 0, AQ_SCALES_TILE_FP32 = 1 } aq_scale_kind;
+
 typedef struct aq_packed {
   int32_t N, K, bN, bK, R, C, T4, T8;
   uint8_t* bitmap;
@@ -85,6 +95,7 @@ typedef struct aq_packed {
   uint8_t* w4;
   int8_t* w8;
   uint16_t* scales;
+  int32_t scale_kind;  /* aq_scale_kind; set by the packers (zero-initialize a struct built by hand) */
 } aq_packed;
 
 /* Index of each buffer in the size array of aq_packed_sizes(). */
@@ -100,6 +111,7 @@ const char* aq_status_str(int status);
  * Host only, no CUDA call.  Byte size of each of the seven packed buffers for
  * an N x K projection with bN x bK tiles of which T4 are INT4.
  * out_bytes: host array of AQ_NUM_BUFS entries.
+ * Either geometry is accepted (bK == 128, or bK == 64 for aq_pack_tiles).
  * Errors: AQ_ERR_ARG (null out_bytes, T4 outside [0, R*C]), AQ_ERR_SHAPE.
  */
 int aq_packed_sizes(int N, int K, int bN, int bK, int T4, size_t* out_bytes);
@@ -144,6 +156,21 @@ int aq_pack_metadata(const uint8_t* map_host, int R, int C, uint8_t* bitmap, int
  */
 int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_t* map, int N, int K, int bN,
             int bK, aq_packed* out, void* stream);
+
+/*
+ * Paper-exact packing (App. B.2, E.2): the same format as aq_pack with ONE
+ * fp32 scale per whole tile (the paper's FP32 tile scale) and 64-wide tiles.
+ *  codes        int8  [N][K] device, as for aq_pack
+ *  tile_scales  fp32  [R][C] device, s^W_{r,j}
+ *  map          uint8 [R][C] device, 1 = INT4 tile, 0 = INT8 tile
+ *  out          as for aq_pack, buffers of aq_packed_sizes(N, K, bN, bK, T4)
+ *               bytes; the scales buffer receives the fp32 tile scales and
+ *               out->scale_kind = AQ_SCALES_TILE_FP32.
+ * Geometry: bN in {64, 128}, bK == 64, N % bN == 0, K % bK == 0.
+ * Offline step: synchronizes `stream`.  Errors as for aq_pack.
+ */
+int aq_pack_tiles(const int8_t* codes, const float* tile_scales, const uint8_t* map, int N, int K, int bN, int bK,
+                  aq_packed* out, void* stream);
 
 /*
  * Float weights -> integer codes and scales for aq_pack (App. B.2, eq. 5-7),
@@ -225,6 +252,50 @@ int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, const float
  */
 int aq_act_group_rows(int M);
 int aq_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream);
+
+/*
+ * Paper-exact activation preparation (App. B.1 eq. 4, App. B.3): the
+ * transformed activations X~ = X V with V = diag(V_0, V_1, ...), one 64 x 64
+ * block per 64 input features, then the groups of aq_quant_act_groups on X~:
+ *   x~[m][64c + k] = sum_{i=0..63} x[m][64c + i] * V_c[i][k]      (fp64)
+ *   per group A of 64 features x b_M rows of X~ (rows zero-padded to M'):
+ *   s = max(max(0, max A) / 127, max(0, -min A) / 128, 1e-12)
+ *   xq = clamp(rint(x~ / s), -128, 127) (fp64 quotient)     sx = (float)s
+ *  x   bf16 [M][ldx] (bits as uint16)
+ *  v   fp32 [K/64][64][64], V_c[i][k] at (c*64 + i)*64 + k; NULL = identity
+ *      (then the result equals aq_quant_act_groups).  The sums are formed in
+ *      fp64; with the paper's transform seeds (entries 0, +-1, +-1/8) and
+ *      bf16 inputs they are exact, so the codes do not depend on the order.
+ *  xq  int8 [M'][K], sx fp32 [M'/b_M][K/64], M' = ceil(M / b_M) * b_M.
+ * Asynchronous.  Errors: AQ_ERR_ARG (null x / xq / sx, M < 1, K < 64,
+ * K % 64, ldx < K), AQ_ERR_CUDA.
+ */
+int aq_paper_quant_act(const uint16_t* x, int M, int K, int ldx, const float* v, int8_t* xq, float* sx,
+                       void* stream);
+
+/*
+ * Paper-exact linear layer (App. E.3 eq. 19, then App. B.1 eq. 4):
+ *   y~[m][n] = sum_j sx[m / b_M][j] * sw[n / bN][j] * P[m][n][j]   (fp32, j ascending)
+ *   P[m][n][j] = sum_{k in tile column j} xq[m][k] * q[n][k]       (exact INT32)
+ *   y[m][r*bN + c] = sum_{i < bN} y~[m][r*bN + i] * U_r[i][c]  (+ bias[r*bN + c])
+ *  w     a projection packed by aq_pack_tiles (bK == 64, per-tile fp32 scales)
+ *  xq    int8 [M'][K] and sx fp32 [M'/b_M][K/64] as aq_paper_quant_act writes them
+ *  u     fp32 [R][bN][bN], U_r[i][c] at (r*bN + i)*bN + c; NULL = identity
+ *  bias  fp32 [N] or NULL
+ *  y     fp32 [M][ldy]; rows m < M are written, nothing else
+ * Any M >= 1 (the CUDA cores compute it; it is the numerics reference of the
+ * paper's own construction, not the per-token layer's fast path).
+ * Asynchronous, no workspace.  Errors: AQ_ERR_ARG (null pointer, M < 1,
+ * ldy < N, a packed struct of the other scale kind), AQ_ERR_SHAPE, AQ_ERR_CUDA.
+ */
+int aq_paper_linear(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* u, const float* bias,
+                    float* y, int ldy, void* stream);
+
+/*
+ * Test entry: the exact integer tile products P[m][n][j] (int32 [M][N][K/64])
+ * of aq_paper_linear, as its kernel forms them.  Errors as aq_paper_linear.
+ */
+int aq_debug_paper_partials(const aq_packed* w, const int8_t* xq, int M, int32_t* P, void* stream);
 
 /*
  * Device scratch bytes a linear call needs for `phase` (aq_phase) at M tokens

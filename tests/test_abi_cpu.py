@@ -52,7 +52,7 @@ def test_packed_sizes_match_oracle(N, K, bN, T4):
 
 @pytest.mark.parametrize("args,status", [
     ((100, 128, 128, 128, 0), -2), ((128, 100, 128, 128, 0), -2), ((128, 128, 32, 128, 0), -2),
-    ((128, 128, 128, 64, 0), -2), ((128, 128, 128, 128, 2), -1), ((128, 128, 128, 128, -1), -1)])
+    ((128, 128, 128, 32, 0), -2), ((128, 128, 128, 128, 2), -1), ((128, 128, 128, 128, -1), -1)])
 def test_packed_sizes_rejects(args, status):
     out = (ctypes.c_size_t * 7)()
     assert aq.lib().aq_packed_sizes(*args, out) == status
@@ -233,3 +233,43 @@ def test_paper_form_activation_quantizer_validation():
     assert f(16, 1, 128, 132, 16, 16, None) == -1     # ldx not a multiple of 8
     assert f(24, 1, 128, 128, 16, 16, None) == -1     # x not 16-byte aligned
     assert f(16, 1, 128, 128, 20, 16, None) == -1     # xq not 8-byte aligned
+
+
+def test_paper_exact_mode_validation():
+    """The paper-exact entries (bK = 64, per-tile fp32 scales) and the per-token
+    layer reject each other's packed structs, before any launch."""
+    L = aq.lib()
+    sizes = aq.aq_packed_sizes(128, 128, 64, 64, 1)
+    assert sizes["w8"] == 3 * 64 * 64 and sizes["w4"] == 64 * 32 and sizes["scales"] >= 4 * 4
+    assert L.aq_pack_tiles(None, 16, 16, 128, 128, 64, 64, None, None) == -1
+    out = aq.AqPackedStruct()
+    assert L.aq_pack_tiles(16, 16, 16, 128, 128, 64, 128, ctypes.byref(out), None) == -2  # bK must be 64
+    assert L.aq_pack_tiles(16, 16, 16, 128, 96, 64, 64, ctypes.byref(out), None) == -2    # K % 64
+    assert L.aq_pack(16, 16, 16, 128, 128, 64, 64, ctypes.byref(out), None) == -2         # per-row form: bK = 128
+    bufs = dict(bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    paper = aq.AqPackedStruct(N=128, K=128, bN=64, bK=64, R=2, C=2, T4=0, T8=4, scale_kind=aq.AQ_SCALES_TILE_FP32,
+                              **bufs)
+    rowform = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1, **bufs)
+    lin = L.aq_paper_linear
+    assert lin(ctypes.byref(rowform), 16, 16, 1, None, None, 16, 128, None) == -1   # fp16 row-scale struct
+    wrong_kind = aq.AqPackedStruct(N=128, K=128, bN=64, bK=64, R=2, C=2, T4=0, T8=4, **bufs)
+    assert lin(ctypes.byref(wrong_kind), 16, 16, 1, None, None, 16, 128, None) == -1
+    bad_geo = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
+                                scale_kind=aq.AQ_SCALES_TILE_FP32, **bufs)
+    assert lin(ctypes.byref(bad_geo), 16, 16, 1, None, None, 16, 128, None) == -2
+    assert lin(ctypes.byref(paper), 16, 16, 0, None, None, 16, 128, None) == -1      # M < 1
+    assert lin(ctypes.byref(paper), 16, 16, 1, None, None, None, 128, None) == -1    # no output
+    assert lin(ctypes.byref(paper), 16, 16, 1, None, None, 16, 100, None) == -1      # ldy < N
+    assert lin(ctypes.byref(paper), 24, 16, 1, None, None, 16, 128, None) == -1      # xq not 16-byte aligned
+    assert L.aq_debug_paper_partials(ctypes.byref(paper), 16, 1, None, None) == -1
+    # the per-token layer refuses a paper-form struct
+    paper128 = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
+                                 scale_kind=aq.AQ_SCALES_TILE_FP32, **bufs)
+    assert L.aq_linear_decode(ctypes.byref(paper128), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_prefill(ctypes.byref(paper128), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_workspace_bytes(0, 1, ctypes.byref(paper128)) == 0
+    q = L.aq_paper_quant_act
+    assert q(None, 1, 128, 128, None, 16, 16, None) == -1
+    assert q(16, 0, 128, 128, None, 16, 16, None) == -1
+    assert q(16, 1, 96, 96, None, 16, 16, None) == -1      # K % 64
+    assert q(16, 1, 128, 120, None, 16, 16, None) == -1    # ldx < K

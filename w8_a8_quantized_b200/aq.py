@@ -25,7 +25,8 @@ EXPORTED = ("aq_status_str", "aq_packed_sizes", "aq_pack_metadata", "aq_pack", "
             "aq_linear_group", "aq_group_workspace_bytes", "aq_workspace_status", "aq_linear_decode_noalloc",
             "aq_quantize_weights", "aq_paper_packed_bytes", "aq_expanded_bytes", "aq_expand_int8",
             "aq_linear_prefill_expanded", "aq_act_group_rows", "aq_quant_act_groups", "aq_measure_i8_peak",
-            "aq_debug_linear_stalled")
+            "aq_debug_linear_stalled", "aq_pack_tiles", "aq_paper_quant_act", "aq_paper_linear",
+            "aq_debug_paper_partials")
 
 
 class AqError(RuntimeError):
@@ -34,9 +35,12 @@ class AqError(RuntimeError):
         super().__init__(f"{what}: {lib().aq_status_str(status).decode()} ({status})")
 
 
+AQ_SCALES_ROW_FP16, AQ_SCALES_TILE_FP32 = 0, 1
+
+
 class AqPackedStruct(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("N", "K", "bN", "bK", "R", "C", "T4", "T8")] + \
-               [(n, ctypes.c_void_p) for n in BUF_NAMES]
+               [(n, ctypes.c_void_p) for n in BUF_NAMES] + [("scale_kind", ctypes.c_int32)]
 
 
 _lib = None
@@ -62,6 +66,14 @@ def lib():
                                    ctypes.POINTER(ctypes.c_int32)]
     L.aq_pack.restype = c_int
     L.aq_pack.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, P, c_void_p]
+    L.aq_pack_tiles.restype = c_int
+    L.aq_pack_tiles.argtypes = [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, P, c_void_p]
+    L.aq_paper_quant_act.restype = c_int
+    L.aq_paper_quant_act.argtypes = [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.aq_paper_linear.restype = c_int
+    L.aq_paper_linear.argtypes = [P, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p]
+    L.aq_debug_paper_partials.restype = c_int
+    L.aq_debug_paper_partials.argtypes = [P, c_void_p, c_int, c_void_p, c_void_p]
     L.aq_quant_act.restype = c_int
     L.aq_paper_packed_bytes.restype = c_int
     L.aq_paper_packed_bytes.argtypes = [c_int, c_int, c_int, c_int, c_int, ctypes.POINTER(c_size_t)]
@@ -186,6 +198,86 @@ def aq_pack(codes: torch.Tensor, scales: torch.Tensor, pmap: torch.Tensor, bN: i
         _check(lib().aq_pack(codes.data_ptr(), scales.data_ptr(), pmap.data_ptr(), N, K, bN, bK,
                              ctypes.byref(w.struct), _stream(dev)), "aq_pack")
     return w
+
+
+def aq_pack_tiles(codes: torch.Tensor, tile_scales: torch.Tensor, pmap: torch.Tensor, bN: int,
+                  bK: int = 64) -> PackedWeights:
+    """Paper-exact packing: codes int8 [N][K], tile_scales float32 [R][C] (one
+    scale per whole tile), pmap uint8 [R][C] (1 = INT4), bK = 64."""
+    _need(codes, "codes", torch.int8)
+    dev = codes.device
+    _need(tile_scales, "tile_scales", torch.float32, dev)
+    _need(pmap, "pmap", torch.uint8, dev)
+    N, K = codes.shape
+    if pmap.dim() != 2 or pmap.shape[0] * bN != N or pmap.shape[1] * bK != K or \
+            tuple(tile_scales.shape) != tuple(pmap.shape):
+        raise ValueError("codes [N][K], tile_scales [R][C] and pmap [R][C] do not agree with the tile shape")
+    T4 = aq_int4_tiles(pmap)
+    w = PackedWeights(N, K, bN, bK, T4, dev)
+    with torch.cuda.device(dev):
+        _check(lib().aq_pack_tiles(codes.data_ptr(), tile_scales.data_ptr(), pmap.data_ptr(), N, K, bN, bK,
+                                   ctypes.byref(w.struct), _stream(dev)), "aq_pack_tiles")
+    return w
+
+
+def aq_paper_quant_act(x: torch.Tensor, v: torch.Tensor = None):
+    """Paper-exact activation preparation: x bf16 [M][ldx], v float32 [K/64][64][64]
+    (V_c blocks; None = identity) -> (xq int8 [M'][K], sx float32 [M'/b_M][K/64])."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 CUDA tensor with unit inner stride")
+    M, K = x.shape
+    if v is not None:
+        _need(v, "v", torch.float32, x.device)
+        if tuple(v.shape) != (K // 64, 64, 64):
+            raise ValueError("v must be float32 [K/64][64][64]")
+    bM = int(lib().aq_act_group_rows(M))
+    Mp = -(-M // bM) * bM
+    xq = torch.empty((Mp, K), dtype=torch.int8, device=x.device)
+    sx = torch.empty((Mp // bM, max(K // 64, 1)), dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(lib().aq_paper_quant_act(x.data_ptr(), M, K, x.stride(0), v.data_ptr() if v is not None else None,
+                                        xq.data_ptr(), sx.data_ptr(), _stream(x.device)), "aq_paper_quant_act")
+    return xq, sx
+
+
+def aq_paper_linear(w: PackedWeights, xq: torch.Tensor, sx: torch.Tensor, M: int, u: torch.Tensor = None,
+                    bias: torch.Tensor = None, out: torch.Tensor = None) -> torch.Tensor:
+    """Paper-exact layer (eq. 19, then Y = Y~ U): w from aq_pack_tiles, (xq, sx)
+    from aq_paper_quant_act, u float32 [R][bN][bN] (None = identity), bias
+    float32 [N] -> y float32 [M][N]."""
+    dev = w.device
+    _need(xq, "xq", torch.int8, dev)
+    _need(sx, "sx", torch.float32, dev)
+    if u is not None:
+        _need(u, "u", torch.float32, dev)
+        if tuple(u.shape) != (w.R, w.bN, w.bN):
+            raise ValueError("u must be float32 [R][bN][bN]")
+    if bias is not None:
+        _need(bias, "bias", torch.float32, dev)
+        if bias.numel() != w.N:
+            raise ValueError("bias must have N elements")
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev)
+    if out.dim() != 2 or out.shape[0] < M or out.shape[1] < w.N or out.stride(1) != 1:
+        raise ValueError("out must be float32 [>= M][>= N] with unit inner stride")
+    with torch.cuda.device(dev):
+        _check(lib().aq_paper_linear(ctypes.byref(w.struct), xq.data_ptr(), sx.data_ptr(), M,
+                                     u.data_ptr() if u is not None else None,
+                                     bias.data_ptr() if bias is not None else None, out.data_ptr(), out.stride(0),
+                                     _stream(dev)), "aq_paper_linear")
+    return out
+
+
+def aq_debug_paper_partials(w: PackedWeights, xq: torch.Tensor, M: int) -> torch.Tensor:
+    """Exact integer tile products of the paper-exact layer: int32 [M][N][K/64]."""
+    dev = w.device
+    _need(xq, "xq", torch.int8, dev)
+    P = torch.zeros((M, w.N, w.C), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().aq_debug_paper_partials(ctypes.byref(w.struct), xq.data_ptr(), M, P.data_ptr(), _stream(dev)),
+               "aq_debug_paper_partials")
+    return P
 
 
 def aq_int4_tiles(pmap: torch.Tensor) -> int:

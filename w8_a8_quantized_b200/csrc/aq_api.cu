@@ -59,6 +59,7 @@ cudaError_t launch_decode_cc(const DecodeProj* projs, int G, int K, const uint16
 
 int validate_packed(const aq_packed* w) {
   if (!w) return AQ_ERR_ARG;
+  if (w->scale_kind != AQ_SCALES_ROW_FP16) return AQ_ERR_ARG;  // the per-token layer's kernels read fp16 row scales
   if (!geometry_ok(w->N, w->K, w->bN, w->bK)) return AQ_ERR_SHAPE;
   if (w->R != w->N / w->bN || w->C != w->K / w->bK) return AQ_ERR_SHAPE;
   if (w->T4 < 0 || w->T8 < 0 || (long long)w->T4 + w->T8 != (long long)w->R * w->C) return AQ_ERR_SHAPE;
@@ -141,7 +142,7 @@ extern "C" const char* aq_status_str(int status) {
 
 extern "C" int aq_packed_sizes(int N, int K, int bN, int bK, int T4, size_t* out) {
   if (!out) return AQ_ERR_ARG;
-  if (!geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
+  if (!geometry_ok(N, K, bN, bK) && !paper_geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
   const long long R = N / bN, C = K / bK, T = R * C;
   if (T4 < 0 || T4 > T) return AQ_ERR_ARG;
   const long long B = (long long)bN * bK;
@@ -207,7 +208,6 @@ extern "C" int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const flo
 }
 
 namespace aq {
-int act_group_rows(int M);
 cudaError_t launch_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx,
                                     cudaStream_t st);
 }  // namespace aq
@@ -242,7 +242,7 @@ extern "C" int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, 
   if (!tmp || ((uintptr_t)tmp & 255)) return AQ_ERR_ARG;
   if (tmp_bytes < expanded_bytes(w)) return AQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  aq_packed e;
+  aq_packed e{};
   cudaError_t err = launch_expand_int8(w, tmp, &e, st);
   if (err == cudaSuccess)
     err = launch_tc(&e, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_PREFILL, st);

@@ -43,6 +43,14 @@ inline bool geometry_ok(int N, int K, int bN, int bK) {
   return N > 0 && K > 0 && (bN == 64 || bN == 128) && bK == kTileK && N % bN == 0 && K % bK == 0 &&
          (long long)N * K < (1ll << 40);
 }
+// The paper-exact mode's tiles: 64 input columns (the activation group width).
+constexpr int kPaperTileK = 64;
+// b_M of App. B.3: activation rows per scale group (1 for a single row, else 16).
+int act_group_rows(int M);
+inline bool paper_geometry_ok(int N, int K, int bN, int bK) {
+  return N > 0 && K > 0 && (bN == 64 || bN == 128) && bK == kPaperTileK && N % bN == 0 && K % bK == 0 &&
+         (long long)N * K < (1ll << 40);
+}
 
 int validate_packed(const aq_packed* w);  // AQ_OK or an error status
 
@@ -95,8 +103,8 @@ size_t prefill_ws_bytes(int M, const aq_packed* w);
 
 // Launchers (defined next to their kernels).  They assume validated arguments.
 cudaError_t launch_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, cudaStream_t st);
-cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, const aq_packed* out,
-                                const uint8_t* map_dev, int* err_dev, cudaStream_t st);
+cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, const float* tile_scales,
+                                const aq_packed* out, const uint8_t* map_dev, int* err_dev, cudaStream_t st);
 // Long-prefill variant: all-INT8 copy of a packed projection in a caller buffer.
 size_t expanded_bytes(const aq_packed* w);
 cudaError_t launch_expand_int8(const aq_packed* w, void* buf, aq_packed* out, cudaStream_t st);

@@ -105,6 +105,7 @@ cudaError_t launch_expand_int8(const aq_packed* w, void* buf, aq_packed* out, cu
   out->w4 = nullptr;
   out->w8 = w8;
   out->scales = w->scales;
+  out->scale_kind = AQ_SCALES_ROW_FP16;
   ExpArgs a{w->bitmap, w->tile_idx, w->w4, w->w8, w->bN, w->R, w->C, w8, idx, off8, off4, bitmap};
   expand_int8_kernel<<<(unsigned)T, kExpThreads, 0, st>>>(a);
   return cudaGetLastError();

@@ -8,7 +8,8 @@
 // Device side: one CTA per logical tile copies the INT8 tile or nibble-packs
 // the INT4 tile (eq. 17: first value in the low nibble) into its precision's
 // buffer, checks INT4 codes are in [-8, 7], and copies the tile's fp16 row
-// scales into logical tile order.
+// scales into logical tile order (or, for the paper-exact form, the tile's one
+// fp32 scale, App. E.2).
 #include <vector>
 
 #include "aq_internal.cuh"
@@ -20,13 +21,14 @@ constexpr int kPackThreads = 256;
 
 struct PackArgs {
   const int8_t* codes;
-  const uint16_t* scales_in;   // [N][C]
+  const uint16_t* scales_in;   // [N][C] fp16 (row scales), or null
+  const float* tile_scales_in; // [R][C] fp32 (tile scales), or null
   const uint8_t* map;          // [R][C]
   const int32_t* tile_idx;     // [R*C]
   uint8_t* w4;
   int8_t* w8;
-  uint16_t* scales_out;        // [R][C][bN]
-  int N, K, bN, R, C;
+  uint16_t* scales_out;        // [R][C][bN] fp16, or [R][C] fp32 bits
+  int N, K, bN, bK, R, C;
   int* err;
 };
 
@@ -35,13 +37,14 @@ __global__ void __launch_bounds__(kPackThreads) pack_payload_kernel(PackArgs a) 
   const int r = t / a.C, j = t % a.C;
   const bool is4 = a.map[t] != 0;
   const size_t p = (size_t)a.tile_idx[t];
-  const int vecs_per_row = kTileK / 16;  // 16-byte vectors of codes per tile row
+  const int bK = a.bK;
+  const int vecs_per_row = bK / 16;  // 16-byte vectors of codes per tile row
   for (int v = threadIdx.x; v < a.bN * vecs_per_row; v += kPackThreads) {
     const int n = v / vecs_per_row, c = v % vecs_per_row;
-    const int8_t* src = a.codes + (size_t)(r * a.bN + n) * a.K + (size_t)j * kTileK + c * 16;
+    const int8_t* src = a.codes + (size_t)(r * a.bN + n) * a.K + (size_t)j * bK + c * 16;
     const int4 q = *reinterpret_cast<const int4*>(src);
     if (!is4) {
-      *reinterpret_cast<int4*>(a.w8 + (p * a.bN + n) * kTileK + c * 16) = q;
+      *reinterpret_cast<int4*>(a.w8 + (p * a.bN + n) * bK + c * 16) = q;
     } else {
       const int8_t* b = reinterpret_cast<const int8_t*>(&q);
       uint32_t packed[2] = {0u, 0u};
@@ -54,19 +57,23 @@ __global__ void __launch_bounds__(kPackThreads) pack_payload_kernel(PackArgs a) 
         packed[i / 4] |= byte << (8 * (i % 4));
       }
       if (bad) atomicExch(a.err, 1);
-      *reinterpret_cast<uint2*>(a.w4 + (p * a.bN + n) * (kTileK / 2) + c * 8) = make_uint2(packed[0], packed[1]);
+      *reinterpret_cast<uint2*>(a.w4 + (p * a.bN + n) * (bK / 2) + c * 8) = make_uint2(packed[0], packed[1]);
     }
   }
-  for (int n = threadIdx.x; n < a.bN; n += kPackThreads)
-    a.scales_out[(size_t)t * a.bN + n] = a.scales_in[(size_t)(r * a.bN + n) * a.C + j];
+  if (a.tile_scales_in != nullptr) {
+    if (threadIdx.x == 0) reinterpret_cast<float*>(a.scales_out)[t] = a.tile_scales_in[t];
+  } else {
+    for (int n = threadIdx.x; n < a.bN; n += kPackThreads)
+      a.scales_out[(size_t)t * a.bN + n] = a.scales_in[(size_t)(r * a.bN + n) * a.C + j];
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, const aq_packed* out,
-                                const uint8_t* map_dev, int* err_dev, cudaStream_t st) {
-  PackArgs a{codes, scales, map_dev, out->tile_idx, out->w4, out->w8, out->scales,
-             out->N, out->K, out->bN, out->R, out->C, err_dev};
+cudaError_t launch_pack_payload(const int8_t* codes, const uint16_t* scales, const float* tile_scales,
+                                const aq_packed* out, const uint8_t* map_dev, int* err_dev, cudaStream_t st) {
+  PackArgs a{codes, scales, tile_scales, map_dev, out->tile_idx, out->w4, out->w8, out->scales,
+             out->N, out->K, out->bN, out->bK, out->R, out->C, err_dev};
   pack_payload_kernel<<<out->R * out->C, kPackThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
@@ -109,17 +116,18 @@ extern "C" int aq_paper_packed_bytes(int R, int C, int T4, int bN, int bK, size_
   return AQ_OK;
 }
 
-extern "C" int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_t* map, int N, int K, int bN,
-                       int bK, aq_packed* out, void* stream) {
+// The host part shared by both packers: labels -> metadata (host), then the
+// payload kernel.  Exactly one of scales (fp16 row scales) and tile_scales (fp32).
+static int pack_common(const int8_t* codes, const uint16_t* scales, const float* tile_scales, const uint8_t* map,
+                       int N, int K, int bN, int bK, aq_packed* out, void* stream) {
   using namespace aq;
-  if (!codes || !scales || !map || !out) return AQ_ERR_ARG;
-  if (!geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
-  if (((uintptr_t)codes & 15) || ((uintptr_t)out->w8 & 15) || ((uintptr_t)out->w4 & 15)) return AQ_ERR_ARG;
   const int R = N / bN, C = K / bK;
   const int T = R * C;
+  if (((uintptr_t)codes & 15) || ((uintptr_t)out->w8 & 15) || ((uintptr_t)out->w4 & 15)) return AQ_ERR_ARG;
   if (out->T4 < 0 || out->T4 > T) return AQ_ERR_ARG;
   if (!out->bitmap || !out->row_off4 || !out->row_off8 || !out->tile_idx || !out->scales) return AQ_ERR_ARG;
   if ((out->T4 > 0 && !out->w4) || (out->T4 < T && !out->w8)) return AQ_ERR_ARG;
+  if (tile_scales != nullptr && ((uintptr_t)out->scales & 3)) return AQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   std::vector<uint8_t> map_h(T), bitmap_h((T + 7) / 8);
@@ -132,6 +140,7 @@ extern "C" int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_
   if (T4 != out->T4) return AQ_ERR_ARG;
 
   out->N = N; out->K = K; out->bN = bN; out->bK = bK; out->R = R; out->C = C; out->T8 = T - T4;
+  out->scale_kind = tile_scales != nullptr ? AQ_SCALES_TILE_FP32 : AQ_SCALES_ROW_FP16;
   if (cudaMemcpyAsync(out->bitmap, bitmap_h.data(), bitmap_h.size(), cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaMemcpyAsync(out->row_off4, off4_h.data(), 4 * (R + 1), cudaMemcpyHostToDevice, st) != cudaSuccess ||
       cudaMemcpyAsync(out->row_off8, off8_h.data(), 4 * (R + 1), cudaMemcpyHostToDevice, st) != cudaSuccess ||
@@ -142,10 +151,24 @@ extern "C" int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_
   if (cudaMalloc(&err_dev, sizeof(int)) != cudaSuccess) return AQ_ERR_CUDA;
   int err_h = 0;
   cudaError_t e = cudaMemsetAsync(err_dev, 0, sizeof(int), st);
-  if (e == cudaSuccess) e = launch_pack_payload(codes, scales, out, map, err_dev, st);
+  if (e == cudaSuccess) e = launch_pack_payload(codes, scales, tile_scales, out, map, err_dev, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(&err_h, err_dev, sizeof(int), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   cudaFree(err_dev);
   if (e != cudaSuccess) return AQ_ERR_CUDA;
   return err_h ? AQ_ERR_RANGE : AQ_OK;
+}
+
+extern "C" int aq_pack(const int8_t* codes, const uint16_t* scales, const uint8_t* map, int N, int K, int bN,
+                       int bK, aq_packed* out, void* stream) {
+  if (!codes || !scales || !map || !out) return AQ_ERR_ARG;
+  if (!aq::geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
+  return pack_common(codes, scales, nullptr, map, N, K, bN, bK, out, stream);
+}
+
+extern "C" int aq_pack_tiles(const int8_t* codes, const float* tile_scales, const uint8_t* map, int N, int K, int bN,
+                             int bK, aq_packed* out, void* stream) {
+  if (!codes || !tile_scales || !map || !out) return AQ_ERR_ARG;
+  if (!aq::paper_geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
+  return pack_common(codes, nullptr, tile_scales, map, N, K, bN, bK, out, stream);
 }
