@@ -27,14 +27,18 @@ __global__ void __launch_bounds__(kGroup) paper_act_kernel(const uint16_t* __res
                                                            const float* __restrict__ v, int8_t* __restrict__ xq,
                                                            float* __restrict__ sx) {
   __shared__ double xs[BM][kGroup];
-  __shared__ float vs[kGroup][kGroup];
+  __shared__ __align__(16) float vs[kGroup][kGroup];
   __shared__ double red[2][2];
   const int k = threadIdx.x, lane = k & 31, wid = k >> 5;
   const int G = K / kGroup;
   const int g = blockIdx.x / G, c = blockIdx.x - g * G;
   pdl_launch_dependents();
-  if (v != nullptr)  // the transform block is a parameter: read it before the wait
-    for (int i = 0; i < kGroup; ++i) vs[i][k] = __ldg(v + ((size_t)c * kGroup + i) * kGroup + k);
+  if (v != nullptr) {  // the transform block is a parameter: read it before the wait, 16 independent 16-byte loads
+    const float4* vb = reinterpret_cast<const float4*>(v + (size_t)c * kGroup * kGroup);
+#pragma unroll
+    for (int i = 0; i < kGroup * kGroup / 4 / kGroup; ++i)
+      reinterpret_cast<float4*>(&vs[0][0])[k + kGroup * i] = __ldg(vb + k + kGroup * i);
+  }
   pdl_wait();  // x may come from the previous kernel; xq / sx may still be read by it
 #pragma unroll
   for (int r = 0; r < BM; ++r) {
@@ -104,22 +108,36 @@ template <int BN, int MT, bool DEBUG>
 __global__ void __launch_bounds__(4 * BN) paper_linear_kernel(const __grid_constant__ PArgs a) {
   static_assert(MT == 1 || MT == 16, "one token, or one 16-row activation group per CTA");
   constexpr int kAcc = MT == 1 ? 1 : MT / 4;
-  extern __shared__ __align__(16) float psm[];  // y~ [MT][BN], then U_r [BN][BN]
+  extern __shared__ __align__(16) float psm[];  // y~ [MT][BN], U_r [BN][BN], tile records [C]
   const int r = blockIdx.x, m0 = blockIdx.y * MT;
   const int n = threadIdx.x >> 2, q = threadIdx.x & 3;
   const int C = a.C, K = a.K;
   const int nrow = r * BN + n;
+  float* yt = psm;            // [MT][BN]
+  float* us = psm + MT * BN;  // [BN][BN]
+  // the tile row's records: physical index with the INT4 label in bit 31, and the
+  // tile scale (divided by 16 for INT4 tiles: their products come as 16 q)
+  int2* rec = reinterpret_cast<int2*>(psm + MT * BN + (a.u != nullptr ? BN * BN : 0));
   pdl_launch_dependents();
+  for (int j = threadIdx.x; j < C; j += 4 * BN) {
+    const int t = r * C + j;
+    const uint32_t is4 = (__ldg(a.bitmap + (t >> 3)) >> (t & 7)) & 1u;
+    const float swt = __ldg(a.sw + t) * (is4 ? 0.0625f : 1.0f);
+    rec[j] = make_int2(__ldg(a.tile_idx + t) | (int)(is4 << 31), __float_as_int(swt));
+  }
+  __syncthreads();
   pdl_wait();
   float acc[kAcc];
 #pragma unroll
   for (int i = 0; i < kAcc; ++i) acc[i] = 0.f;
   const int8_t* xbase = a.xq + (size_t)m0 * K + 16 * q;
   const float* sxrow = a.sx + (size_t)(m0 / a.bM) * C;  // one activation scale row per CTA (MT <= b_M)
+  constexpr int kUnroll = MT == 1 ? 4 : 1;  // (16 token partials per tile leave no registers for more)
+#pragma unroll kUnroll
   for (int j = 0; j < C; ++j) {
-    const int t = r * C + j;
-    const uint32_t is4 = (__ldg(a.bitmap + (t >> 3)) >> (t & 7)) & 1u;
-    const size_t prow = (size_t)__ldg(a.tile_idx + t) * BN + n;
+    const int2 rj = rec[j];
+    const uint32_t is4 = (uint32_t)rj.x >> 31;
+    const size_t prow = (size_t)(rj.x & 0x7fffffff) * BN + n;
     int part[MT];
     if (!is4) {
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(a.w8 + prow * kGroup + 16 * q));
@@ -174,16 +192,13 @@ __global__ void __launch_bounds__(4 * BN) paper_linear_kernel(const __grid_const
           a.P[((size_t)m * a.N + nrow) * C + j] = is4 ? (prod[i] >> 4) : prod[i];  // 16 q products / 16, exact
       }
     } else {
-      const float swt = __ldg(a.sw + t) * (is4 ? 0.0625f : 1.0f);
-      const float f = swt * __ldg(sxrow + j);
+      const float f = __int_as_float(rj.y) * __ldg(sxrow + j);
 #pragma unroll
       for (int i = 0; i < kAcc; ++i) acc[i] = fmaf((float)prod[i], f, acc[i]);  // |prod| < 2^24: exact
     }
   }
   if constexpr (DEBUG) return;
 
-  float* yt = psm;            // [MT][BN]
-  float* us = psm + MT * BN;  // [BN][BN]
   if constexpr (MT == 1) {
     if (q == 0) yt[n] = acc[0];
   } else {
@@ -207,10 +222,13 @@ __global__ void __launch_bounds__(4 * BN) paper_linear_kernel(const __grid_const
   }
 }
 
+constexpr int kPaperSmemAttr = 200 * 1024;  // >= every launch's request (the tile records take 8 bytes per tile)
+
 template <int BN, int MT, bool DEBUG>
 cudaError_t launch_paper_t(const PArgs& a, dim3 grid, cudaStream_t st) {
-  const size_t smem = DEBUG ? 0 : (size_t)(MT * BN + (a.u ? BN * BN : 0)) * sizeof(float);
-  cudaError_t e = ensure_smem_attr<paper_linear_kernel<BN, MT, DEBUG>>((int)((MT * BN + BN * BN) * sizeof(float)));
+  const size_t smem = (size_t)(MT * BN + (a.u ? BN * BN : 0)) * sizeof(float) + (size_t)a.C * sizeof(int2);
+  if (smem > (size_t)kPaperSmemAttr) return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_attr<paper_linear_kernel<BN, MT, DEBUG>>(kPaperSmemAttr);
   if (e != cudaSuccess) return e;
   return launch_pdl(paper_linear_kernel<BN, MT, DEBUG>, grid, dim3(4 * BN), smem, st, a);
 }
