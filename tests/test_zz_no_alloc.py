@@ -63,7 +63,8 @@ def test_noalloc_back_to_back_different_shapes():
 
 
 def test_noalloc_rejects_scratch_beyond_limit():
-    _, _, w, xq, sx = _case(3072, 3072, 64, 4200)
+    # a long-K projection at 64 tokens keeps split-K partial sums beyond the 4 MiB scratch
+    _, _, w, xq, sx = _case(6144, 16384, 64, 4200)
     assert aq.aq_workspace_bytes(aq.AQ_PHASE_DECODE, 64, w) > 4 << 20
     with pytest.raises(aq.AqError) as e:
         aq.aq_linear_decode_noalloc(w, xq, sx)

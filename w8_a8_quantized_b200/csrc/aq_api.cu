@@ -71,6 +71,8 @@ int validate_packed(const aq_packed* w) {
 
 static int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 static constexpr int kMaxSplits = 8;
+// Input tiles per split at least (see plan_decode).
+static int min_split_tiles(int M) { return M <= 16 ? 5 : M <= 32 ? 8 : 20; }
 
 // Fusing the activation preparation into every CTA of the CUDA-core decode
 // kernel pays off for 1-2 tokens; from 4 tokens on, one preparation kernel plus
@@ -96,9 +98,16 @@ DecodePlan plan_decode(int M, const aq_packed* w) {
     p.kernel = 1;
     p.rows = 128;
     p.blocks = ceil_div(w->R, 128 / w->bN);
-    // one wave (blocks x S <= SMs), and at most kMaxSplits: the CTA that sums a
-    // unit's splits pays one round of L2 latency per split
-    p.S = std::max(1, std::min(std::min(w->C, kMaxSplits), num_sms() / p.blocks));
+    // One wave (blocks x S <= SMs), at most kMaxSplits, and at least
+    // min_split_tiles(M) input tiles per split: splitting shortens every CTA's
+    // tile chain but costs the unit a round of partial sums that grows with the
+    // token count.  From 32 tokens on, a projection whose row blocks alone fill
+    // a third of the GPU is not split.  (Measured per projection shape at 16, 32
+    // and 64 tokens for 1-8 splits: this rule is within 4% of the best split
+    // count on every shape of the 3B- and 8B-class models.)
+    const int sms = num_sms();
+    p.S = std::max(1, std::min(std::min(w->C / min_split_tiles(M), kMaxSplits), sms / p.blocks));
+    if (M >= 32 && 3 * p.blocks >= sms) p.S = 1;
   }
   return p;
 }
