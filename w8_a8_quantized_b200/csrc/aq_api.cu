@@ -95,20 +95,26 @@ DecodePlan plan_decode(int M, const aq_packed* w) {
     p.blocks = w->N / kRowsPerCta;
     p.S = 1;
   } else {
-    p.kernel = 1;
-    p.rows = 128;
-    p.blocks = ceil_div(w->R, 128 / w->bN);
-    // One wave (blocks x S <= SMs), at most kMaxSplits, and at least
-    // min_split_tiles(M) input tiles per split: splitting shortens every CTA's
-    // tile chain but costs the unit a round of partial sums that grows with the
-    // token count.  From 32 tokens on, a projection whose row blocks alone fill
-    // a third of the GPU is not split.  (Measured per projection shape at 16, 32
-    // and 64 tokens for 1-8 splits: this rule is within 4% of the best split
-    // count on every shape of the 3B- and 8B-class models.)
-    const int sms = num_sms();
-    p.S = std::max(1, std::min(std::min(w->C / min_split_tiles(M), kMaxSplits), sms / p.blocks));
-    if (M >= 32 && 3 * p.blocks >= sms) p.S = 1;
+    p = plan_tc_decode(M, ceil_div(w->R, 128 / w->bN), w->C);
   }
+  return p;
+}
+
+DecodePlan plan_tc_decode(int M, int blocks, int C) {
+  DecodePlan p;
+  p.kernel = 1;
+  p.rows = 128;
+  p.blocks = blocks;
+  // One wave (blocks x S <= SMs), at most kMaxSplits, and at least
+  // min_split_tiles(M) input tiles per split: splitting shortens every CTA's
+  // tile chain but costs the unit a round of partial sums that grows with the
+  // token count.  From 32 tokens on, a launch whose row blocks alone fill a
+  // third of the GPU is not split.  (Measured per projection shape at 16, 32 and
+  // 64 tokens for 1-8 splits: this rule is within 4% of the best split count on
+  // every shape of the 3B- and 8B-class models.)
+  const int sms = num_sms();
+  p.S = std::max(1, std::min(std::min(C / min_split_tiles(M), kMaxSplits), sms / p.blocks));
+  if (M >= 32 && 3 * p.blocks >= sms) p.S = 1;
   return p;
 }
 
@@ -316,11 +322,39 @@ static bool group_fused(int phase, const aq_packed* const* w, int G, int M) {
 
 static size_t align256(size_t b) { return (b + 255) / 256 * 256; }
 
+// Decode: one tensor-core launch over all members' rows when every member would
+// run on the tensor cores alone, with the same tile shape and whole 128-row
+// blocks per member (q/k/v and gate/up at 32 and 64 tokens: 31-32% less time per
+// 3B-class step; prefill gains nothing from it, its launches are long).
+static bool group_tc(int phase, const aq_packed* const* w, int G, int M) {
+  if (G < 2 || phase != AQ_PHASE_DECODE || M > kMaxDecodeM) return false;
+  for (int g = 0; g < G; ++g) {
+    if (w[g]->bN != w[0]->bN || w[g]->N % 128 != 0) return false;
+    if (phase == AQ_PHASE_DECODE && plan_decode(M, w[g]).kernel != 1) return false;
+  }
+  return true;
+}
+
+// Workspace of the grouped tensor-core launch (header, split counters, split partial sums).
+static size_t group_tc_ws_bytes(int phase, int M, const aq_packed* const* w, int G) {
+  int blocks = 0, N = 0;
+  for (int g = 0; g < G; ++g) {
+    blocks += w[g]->N / 128;
+    N += w[g]->N;
+  }
+  if (phase != AQ_PHASE_DECODE) return kWsHeader + counters_bytes(blocks);
+  const DecodePlan p = plan_tc_decode(M, blocks, w[0]->C);
+  size_t b = kWsHeader + counters_bytes(p.blocks);
+  if (p.S > 1) b += (size_t)p.S * ((M + 3) & ~3) * N * sizeof(float);
+  return b;
+}
+
 static size_t group_ws_bytes(int phase, int M, const aq_packed* const* w, int G) {
   if (group_fused(phase, w, G, M)) return kWsHeader;
   size_t lin = 0;
   for (int g = 0; g < G; ++g)
     lin = std::max(lin, phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w[g]) : prefill_ws_bytes(M, w[g]));
+  if (group_tc(phase, w, G, M)) lin = std::max(lin, group_tc_ws_bytes(phase, M, w, G));
   // the linear workspace (header first), then the prepared activations
   return align256(lin) + align256((size_t)M * w[0]->K) + align256((size_t)M * sizeof(float));
 }
@@ -371,6 +405,7 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   size_t lin = 0;
   for (int g = 0; g < G; ++g)
     lin = std::max(lin, phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w[g]) : prefill_ws_bytes(M, w[g]));
+  if (group_tc(phase, w, G, M)) lin = std::max(lin, group_tc_ws_bytes(phase, M, w, G));
   char* base = static_cast<char*>(ws);
   int8_t* xq = reinterpret_cast<int8_t*>(base + align256(lin));
   float* sx = reinterpret_cast<float*>(base + align256(lin) + align256((size_t)M * K));
@@ -379,6 +414,10 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
     DecodeProj d[kMaxGroup];
     for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
     e = launch_decode_cc(d, G, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
+    return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
+  }
+  if (e == cudaSuccess && group_tc(phase, w, G, M)) {  // one tensor-core launch over all members' rows
+    e = launch_tc_group(w, G, bias, y, ldy, xq, sx, M, ydtype, ws, phase, st);
     return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
   }
   for (int g = 0; e == cudaSuccess && g < G; ++g) {

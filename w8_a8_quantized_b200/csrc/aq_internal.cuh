@@ -98,6 +98,8 @@ struct DecodePlan {
   int blocks;   // number of CTA row blocks
 };
 DecodePlan plan_decode(int M, const aq_packed* w);
+// The tensor-core part of the decode plan for `blocks` 128-row blocks of C input tiles.
+DecodePlan plan_tc_decode(int M, int blocks, int C);
 size_t decode_ws_bytes(int M, const aq_packed* w);
 size_t prefill_ws_bytes(int M, const aq_packed* w);
 
@@ -110,6 +112,11 @@ size_t expanded_bytes(const aq_packed* w);
 cudaError_t launch_expand_int8(const aq_packed* w, void* buf, aq_packed* out, cudaStream_t st);
 cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
                       int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st);
+// One tensor-core launch over G projections that share xq (their 128-row blocks
+// concatenated; same K and bN; every member's rows a multiple of 128).
+cudaError_t launch_tc_group(const aq_packed* const* w, int G, const float* const* bias, void* const* y,
+                            const int* ldy, const int8_t* xq, const float* sx, int M, int ydtype, void* ws, int phase,
+                            cudaStream_t st);
 // Test form of launch_tc: every bounded wait gives up after wait_ns and the
 // weight producer stops after `stop_after` tiles (so later stages never fill).
 cudaError_t launch_tc_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, void* y, int ldy,

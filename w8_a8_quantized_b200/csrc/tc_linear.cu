@@ -50,6 +50,11 @@
 // cores, as many cycles per SM as the INT8 MMA itself; the float2 forms
 // halve the issue slots it takes so tensor-memory work fits beside it.
 //
+// A launch may cover up to kMaxGroup projections that read the same input
+// (q/k/v, gate/up: AlignQuant Sec. 3.3 "Shared activation preparation", App.
+// E.4): their 128-row blocks are concatenated, each block belonging to one
+// member (every member's rows are a multiple of 128 then), and each role looks
+// up the member of the block it works on.
 // A work unit is (128-row block of output features, NT-token block, split of
 // the input tiles).  Split partial sums go to the workspace; the CTA that
 // finishes a unit last sums all splits in increasing split order.
@@ -121,19 +126,27 @@ constexpr uint32_t kAccBias = 0x4B400000u;  // fp32 bit pattern of 12582912 = 1.
 constexpr float kAccBiasF = 12582912.0f;
 constexpr unsigned long long kAbortGraceNs = 200000;  // copies in flight when a CTA gives up
 
-struct TcArgs {
+// One projection of the launch.
+struct TcMember {
   const uint8_t* bitmap;
   const int32_t* tile_idx;
   const uint16_t* scales;
-  int N, K, bN, R, C, T4, T8;
+  const float* bias;
+  void* y;
+  int ldy, N, R, T4, T8;
+  int rb0;  // first 128-row block of the member among the launch's blocks
+};
+
+struct TcArgs {
+  TcMember mem[kMaxGroup];
+  int G;
+  int N, K, bN, C;  // N: rows of all members (the split partial sums span them)
   int tpb;     // tile rows per 128-row block (1 for bN = 128, 2 for bN = 64)
   int nrb;     // number of 128-row blocks
   int M, ntb;  // tokens, token blocks
   int S, units;
   const float* sx;
-  const float* bias;
-  void* y;
-  int ydtype, ldy;
+  int ydtype;
   void* ws;
   float* partial;  // [S][N][Mp], Mp = M rounded up to a multiple of 4
   int* counters;   // [nrb * ntb]
@@ -145,6 +158,22 @@ struct TcArgs {
 
 struct Unit {
   int rb, tb, s, j0, j1;
+};
+
+// Member owning 128-row block rb (member 0 in a single-projection kernel).
+template <bool GROUPED>
+__device__ __forceinline__ int member_of(const TcArgs& a, int rb) {
+  if constexpr (!GROUPED) return 0;
+  int g = 0;
+  while (g + 1 < a.G && rb >= a.mem[g + 1].rb0) ++g;
+  return g;
+}
+
+// Tensor maps of the launch: each member's INT8 and INT4 payloads, and the activations.
+struct TcMaps {
+  CUtensorMap w8[kMaxGroup];
+  CUtensorMap w4[kMaxGroup];
+  CUtensorMap x;
 };
 
 __device__ __forceinline__ Unit unit_of(const TcArgs& a, int u) {
@@ -188,8 +217,8 @@ struct TileIter {
 // issue the tile's copies.
 struct MetaRec {
   uint32_t a_row0, a_row1;  // first row of each sub-tile's weight tile in its precision's buffer
-  uint32_t sizes;           // INT8 KiB | INT4 KiB << 8 | kinds << 28 (copy sizes are whole KiB)
-  uint32_t sc_off;          // element offset of sub-tile 0's scales (sub-tile 1: + C * bN)
+  uint32_t sizes;           // INT8 KiB | INT4 KiB << 8 | member << 16 | kinds << 28 (copy sizes are whole KiB)
+  uint32_t sc_off;          // element offset of sub-tile 0's scales in its member (sub-tile 1: + C * bN)
 };
 // kinds: bits 0-1 INT4 label of sub-tile 0/1, bits 2-3 sub-tile 0/1 exists
 // (the last 128-row block of a bN = 64 layer may hold one tile row only).
@@ -266,8 +295,8 @@ constexpr int chunk_cols(int kCols, int lim) {
 // increasing), scaled by the token scales, plus bias, stored.  CH columns at a
 // time with the loads of all (at most SMAX) splits in flight together.
 template <int kCols, int CH, int SMAX>
-__device__ __forceinline__ void reduce_splits(const TcArgs& a, const float* prow, size_t sstride, int mcol0, int n,
-                                              float bias_n) {
+__device__ __forceinline__ void reduce_splits(const TcArgs& a, const TcMember& mb, const float* prow, size_t sstride,
+                                              int mcol0, int n, float bias_n) {
   static_assert(kCols % CH == 0 && CH % 4 == 0, "reduction chunks");
   const bool sx_vec = ((uintptr_t)a.sx & 15) == 0;
 #pragma unroll 1
@@ -303,17 +332,19 @@ __device__ __forceinline__ void reduce_splits(const TcArgs& a, const float* prow
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        if (m0 + e < a.M) store_y(a.y, a.ydtype, (size_t)(m0 + e) * a.ldy + n, fmaf(xs[e], sv[e], bias_n));
+        if (m0 + e < a.M) store_y(mb.y, a.ydtype, (size_t)(m0 + e) * mb.ldy + n, fmaf(xs[e], sv[e], bias_n));
     }
   }
 }
 
 // MODE: 0 = outputs written directly (one split), 1 = split-K partial sums
 // reduced by the last CTA of each unit group, 2 = exact tile products only.
-template <int NT, int MODE>
+// GROUPED: the launch covers several projections (decode only); single-projection
+// kernels compile without the member lookups, which cost the prefill kernels
+// registers (3-9% of their rate when always present).
+template <int NT, int MODE, bool GROUPED>
 __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
-    tc_linear_kernel(const __grid_constant__ CUtensorMap tm_w8, const __grid_constant__ CUtensorMap tm_w4,
-                     const __grid_constant__ CUtensorMap tm_x, const TcArgs a) {
+    tc_linear_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcArgs a) {
   using Sh = TcShape<NT>;
   constexpr int S_ = Sh::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -370,9 +401,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
     *abort_flag = 0;
     *never_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&tm_x);
-    if (a.T8 > 0) prefetch_tmap(&tm_w8);
-    if (a.T4 > 0) prefetch_tmap(&tm_w4);
+    prefetch_tmap(&maps.x);
+    for (int g = 0; g < a.G; ++g) {
+      if (a.mem[g].T8 > 0) prefetch_tmap(&maps.w8[g]);
+      if (a.mem[g].T4 > 0) prefetch_tmap(&maps.w4[g]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Sh::kTmemCols);
@@ -410,18 +443,22 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
           break;
         }
         const uint32_t kinds = rec.sizes >> 28;
+        const uint32_t mg = GROUPED ? (rec.sizes >> 16) & 0xFu : 0u;  // member of the tile's row block
+        const uint16_t* scales = a.mem[mg].scales;
+        const CUtensorMap* m8 = &maps.w8[mg];
+        const CUtensorMap* m4 = &maps.w4[mg];
         const uint32_t sc_bytes = (kinds & 8) ? 4u * a.bN : 2u * a.bN;  // fp16 row scales of the tile's sub-tiles
         stage_info[sr.i] = kinds;  // read by the transform warps after `staged`
         mbar_arrive_expect_tx(&full[sr.i], (rec.sizes & 0xFFu) << 10);
         mbar_arrive_expect_tx(&staged[sr.i], (((rec.sizes >> 8) & 0xFFu) << 10) + sc_bytes);
         uint8_t* scd = stage_sc + sr.i * 256;
-        bulk_load(scd, a.scales + rec.sc_off, a.bN * 2, &staged[sr.i]);
-        if (kinds & 8) bulk_load(scd + a.bN * 2, a.scales + rec.sc_off + (uint32_t)a.C * a.bN, a.bN * 2, &staged[sr.i]);
-        if (kinds & 1) tma_load_2d(stage_g(sr.i), &tm_w4, 0, rec.a_row0, &staged[sr.i]);
-        else tma_load_2d(stage_a(sr.i), &tm_w8, 0, rec.a_row0, &full[sr.i]);
+        bulk_load(scd, scales + rec.sc_off, a.bN * 2, &staged[sr.i]);
+        if (kinds & 8) bulk_load(scd + a.bN * 2, scales + rec.sc_off + (uint32_t)a.C * a.bN, a.bN * 2, &staged[sr.i]);
+        if (kinds & 1) tma_load_2d(stage_g(sr.i), m4, 0, rec.a_row0, &staged[sr.i]);
+        else tma_load_2d(stage_a(sr.i), m8, 0, rec.a_row0, &full[sr.i]);
         if (kinds & 8) {
-          if (kinds & 2) tma_load_2d(stage_g(sr.i) + a.bN * (kTileK / 2), &tm_w4, 0, rec.a_row1, &staged[sr.i]);
-          else tma_load_2d(stage_a(sr.i) + a.bN * kTileK, &tm_w8, 0, rec.a_row1, &full[sr.i]);
+          if (kinds & 2) tma_load_2d(stage_g(sr.i) + a.bN * (kTileK / 2), m4, 0, rec.a_row1, &staged[sr.i]);
+          else tma_load_2d(stage_a(sr.i) + a.bN * kTileK, m8, 0, rec.a_row1, &full[sr.i]);
         }
         sr.next<S_>();
       }
@@ -480,13 +517,16 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       const int ms = g % kMetaSlots;
       if (!mbar_wait(&meta_empty[ms], ((g / kMetaSlots) & 1) ^ 1, abort_flag, a.wait_ns)) { fail(7); break; }
       uint32_t kinds = 0, bytes8 = 0, bytes4 = 0, row[2] = {0, 0};
+      const int mg = member_of<GROUPED>(a, x.rb);
+      const TcMember& mb = a.mem[mg];
+      const int lrb = GROUPED ? x.rb - mb.rb0 : x.rb;  // row block inside the member
       for (int sub = 0; sub < a.tpb; ++sub) {
-        const int r = x.rb * a.tpb + sub;
-        if (r < a.R) {
+        const int r = lrb * a.tpb + sub;
+        if (r < mb.R) {
           const int t = r * a.C + j;
-          const uint32_t is4 = __ldg(a.bitmap + (t >> 3)) >> (t & 7) & 1;
+          const uint32_t is4 = __ldg(mb.bitmap + (t >> 3)) >> (t & 7) & 1;
           kinds |= (1u << (2 + sub)) | (is4 << sub);
-          row[sub] = (uint32_t)__ldg(a.tile_idx + t) * a.bN;
+          row[sub] = (uint32_t)__ldg(mb.tile_idx + t) * a.bN;
           if (is4) bytes4 += a.bN * (kTileK / 2);
           else bytes8 += a.bN * kTileK;
         }
@@ -494,8 +534,8 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
       MetaRec rec;
       rec.a_row0 = row[0];
       rec.a_row1 = row[1];
-      rec.sizes = (bytes8 >> 10) | ((bytes4 >> 10) << 8) | (kinds << 28);
-      rec.sc_off = (uint32_t)((x.rb * a.tpb) * a.C + j) * a.bN;
+      rec.sizes = (bytes8 >> 10) | ((bytes4 >> 10) << 8) | ((uint32_t)mg << 16) | (kinds << 28);
+      rec.sc_off = (uint32_t)((lrb * a.tpb) * a.C + j) * a.bN;
       meta[ms] = rec;
       mbar_arrive(&meta_full[ms]);
       g += kMetaSlots;
@@ -515,7 +555,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
           break;
         }
         mbar_arrive_expect_tx(&full[sr.i], Sh::kB);
-        tma_load_2d(stage_b(sr.i), &tm_x, bi.j * kTileK, bi.x.tb * NT, &full[sr.i]);
+        tma_load_2d(stage_b(sr.i), &maps.x, bi.j * kTileK, bi.x.tb * NT, &full[sr.i]);
         sr.next<S_>();
       }
       if (!ok || *abort_flag) abort_grace();
@@ -595,14 +635,16 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
     uint32_t g = 0, sync_phase = 0;
     for (int u = blockIdx.x; ok && u < a.units; u += gridDim.x) {
       const Unit x = unit_of(a, u);
-      const int n = x.rb * 128 + row;  // output feature of this thread
-      const bool rvalid = n < a.N;
+      const TcMember& mb = a.mem[member_of<GROUPED>(a, x.rb)];
+      const int n = x.rb * 128 + row;  // row among all members' rows (split partial sums)
+      const int nl = GROUPED ? (x.rb - mb.rb0) * 128 + row : n;  // output feature of this thread in its member
+      const bool rvalid = nl < mb.N;
       const int mcol0 = x.tb * NT + cg * kCols;  // first token of this thread's columns
       // bias of this row and the token scales of the warp's columns, copied
       // into shared memory now and read at the end of the unit
       if constexpr (MODE != 2) {
-        const bool has_b = rvalid && a.bias != nullptr;
-        cp_async4(pre_bias + et, has_b ? a.bias + n : a.sx, has_b ? 4u : 0u);
+        const bool has_b = rvalid && mb.bias != nullptr;
+        cp_async4(pre_bias + et, has_b ? mb.bias + nl : a.sx, has_b ? 4u : 0u);
         for (int c = lane; c < kCols; c += 32) {
           const bool has_s = mcol0 + c < a.M;
           cp_async4(pre_sx + ew * kCols + c, has_s ? a.sx + mcol0 + c : a.sx, has_s ? 4u : 0u);
@@ -653,7 +695,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
             if constexpr (MODE == 2) {
               // INT4 label read back from the bitmap (debug path only)
               const int tt = (n / a.bN) * a.C + j + k;
-              const bool t4 = rvalid && ((__ldg(a.bitmap + (tt >> 3)) >> (tt & 7)) & 1);
+              const bool t4 = rvalid && ((__ldg(mb.bitmap + (tt >> 3)) >> (tt & 7)) & 1);
 #pragma unroll
               for (int e = 0; e < kL; ++e) {
                 const int m = mcol0 + c0 + e;
@@ -690,7 +732,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
         const float4* sxv = reinterpret_cast<const float4*>(pre_sx + ew * kCols);
         const int mlim = a.M - mcol0;  // columns of this thread that exist
         if (rvalid && a.ydtype == AQ_F32) {
-          float* yp = reinterpret_cast<float*>(a.y) + (size_t)mcol0 * a.ldy + n;
+          float* yp = reinterpret_cast<float*>(mb.y) + (size_t)mcol0 * mb.ldy + nl;
 #pragma unroll
           for (int i4 = 0; i4 < kCols / 4; ++i4) {
             const float4 s4 = sxv[i4];
@@ -698,11 +740,11 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int i = 4 * i4 + k;
-              if (i < mlim) yp[(size_t)i * a.ldy] = fmaf(sv[k], i & 1 ? acc[i / 2].y : acc[i / 2].x, bias_n);
+              if (i < mlim) yp[(size_t)i * mb.ldy] = fmaf(sv[k], i & 1 ? acc[i / 2].y : acc[i / 2].x, bias_n);
             }
           }
         } else if (rvalid) {
-          __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(a.y) + (size_t)mcol0 * a.ldy + n;
+          __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(mb.y) + (size_t)mcol0 * mb.ldy + nl;
 #pragma unroll
           for (int i4 = 0; i4 < kCols / 4; ++i4) {
             const float4 s4 = sxv[i4];
@@ -711,7 +753,7 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
             for (int k = 0; k < 4; ++k) {
               const int i = 4 * i4 + k;
               if (i < mlim)
-                yp[(size_t)i * a.ldy] = __float2bfloat16_rn(fmaf(sv[k], i & 1 ? acc[i / 2].y : acc[i / 2].x, bias_n));
+                yp[(size_t)i * mb.ldy] = __float2bfloat16_rn(fmaf(sv[k], i & 1 ? acc[i / 2].y : acc[i / 2].x, bias_n));
             }
           }
         }
@@ -745,9 +787,9 @@ __global__ void __maxnreg__(TcShape<NT>::kMaxRegs)
           // the loads of every split for a chunk of columns are issued before any
           // of them is summed, then the splits are added in increasing order;
           // chunks are as wide as 64 values in flight allow
-          if (a.S <= 2) reduce_splits<kCols, chunk_cols(kCols, 32), 2>(a, prow, sstride, mcol0, n, bias_n);
-          else if (a.S <= 4) reduce_splits<kCols, chunk_cols(kCols, 16), 4>(a, prow, sstride, mcol0, n, bias_n);
-          else reduce_splits<kCols, chunk_cols(kCols, 8), kMaxTcSplits>(a, prow, sstride, mcol0, n, bias_n);
+          if (a.S <= 2) reduce_splits<kCols, chunk_cols(kCols, 32), 2>(a, mb, prow, sstride, mcol0, nl, bias_n);
+          else if (a.S <= 4) reduce_splits<kCols, chunk_cols(kCols, 16), 4>(a, mb, prow, sstride, mcol0, nl, bias_n);
+          else reduce_splits<kCols, chunk_cols(kCols, 8), kMaxTcSplits>(a, mb, prow, sstride, mcol0, nl, bias_n);
         }
         if (ew == 0 && lane == 0) a.counters[x.rb * a.ntb + x.tb] = 0;
       }
@@ -795,36 +837,53 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT, int MODE>
-cudaError_t launch_nt(const aq_packed* w, const int8_t* xq, TcArgs a, int grid, cudaStream_t st) {
+template <int NT, int MODE, bool GROUPED = false>
+cudaError_t launch_nt(const aq_packed* const* w, const int8_t* xq, const TcArgs& a, int grid, cudaStream_t st) {
   using Sh = TcShape<NT>;
-  cudaError_t e = ensure_smem_attr<tc_linear_kernel<NT, MODE>>(Sh::kSmemBytes);
+  cudaError_t e = ensure_smem_attr<tc_linear_kernel<NT, MODE, GROUPED>>(Sh::kSmemBytes);
   if (e != cudaSuccess) return e;
-  CUtensorMap m8, m4, mx;
-  memset(&m8, 0, sizeof(m8));
-  memset(&m4, 0, sizeof(m4));
-  if (w->T8 > 0 && !make_map(&m8, w->w8, kTileK, (uint64_t)w->T8 * w->bN, kTileK, w->bN, true))
-    return cudaErrorInvalidValue;
-  if (w->T4 > 0 && !make_map(&m4, w->w4, kTileK / 2, (uint64_t)w->T4 * w->bN, kTileK / 2, w->bN, false))
-    return cudaErrorInvalidValue;
-  if (!make_map(&mx, xq, w->K, a.M, kTileK, NT, true)) return cudaErrorInvalidValue;
-  return launch_pdl(tc_linear_kernel<NT, MODE>, dim3(grid), dim3(Sh::kThreads), (size_t)Sh::kSmemBytes, st, m8, m4, mx, a);
+  TcMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  for (int g = 0; g < a.G; ++g) {
+    if (w[g]->T8 > 0 && !make_map(&maps.w8[g], w[g]->w8, kTileK, (uint64_t)w[g]->T8 * w[g]->bN, kTileK, w[g]->bN, true))
+      return cudaErrorInvalidValue;
+    if (w[g]->T4 > 0 &&
+        !make_map(&maps.w4[g], w[g]->w4, kTileK / 2, (uint64_t)w[g]->T4 * w[g]->bN, kTileK / 2, w[g]->bN, false))
+      return cudaErrorInvalidValue;
+  }
+  if (!make_map(&maps.x, xq, w[0]->K, a.M, kTileK, NT, true)) return cudaErrorInvalidValue;
+  return launch_pdl(tc_linear_kernel<NT, MODE, GROUPED>, dim3(grid), dim3(Sh::kThreads), (size_t)Sh::kSmemBytes, st,
+                    maps, a);
 }
 
 }  // namespace
 
-static cudaError_t launch_tc_impl(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
-                                  void* y, int ydtype, int ldy, void* ws, int32_t* P, int phase,
-                                  unsigned long long wait_ns, int stop_after, cudaStream_t st) {
+// G members share K and bN; with G > 1 every member's rows are a multiple of 128.
+static cudaError_t launch_tc_impl(const aq_packed* const* w, int G, const float* const* bias, void* const* y,
+                                  const int* ldy, const int8_t* xq, const float* sx, int M, int ydtype, void* ws,
+                                  int32_t* P, int phase, unsigned long long wait_ns, int stop_after, cudaStream_t st) {
+  if (G < 1 || G > kMaxGroup || (P != nullptr && G != 1)) return cudaErrorInvalidValue;
   TcArgs a;
+  memset(&a, 0, sizeof(a));
   a.wait_ns = wait_ns;
   a.stop_after = stop_after;
-  a.bitmap = w->bitmap; a.tile_idx = w->tile_idx; a.scales = w->scales;
-  a.N = w->N; a.K = w->K; a.bN = w->bN; a.R = w->R; a.C = w->C; a.T4 = w->T4; a.T8 = w->T8;
-  a.tpb = 128 / w->bN;
-  a.nrb = (w->R + a.tpb - 1) / a.tpb;
+  a.G = G;
+  a.K = w[0]->K; a.bN = w[0]->bN; a.C = w[0]->C;
+  a.tpb = 128 / a.bN;
+  int rb = 0;
+  for (int g = 0; g < G; ++g) {
+    if (w[g]->K != a.K || w[g]->bN != a.bN || (G > 1 && w[g]->N % 128 != 0)) return cudaErrorInvalidValue;
+    TcMember& m = a.mem[g];
+    m.bitmap = w[g]->bitmap; m.tile_idx = w[g]->tile_idx; m.scales = w[g]->scales;
+    m.bias = bias ? bias[g] : nullptr; m.y = y ? y[g] : nullptr; m.ldy = ldy ? ldy[g] : w[g]->N;
+    m.N = w[g]->N; m.R = w[g]->R; m.T4 = w[g]->T4; m.T8 = w[g]->T8;
+    m.rb0 = rb;
+    rb += (w[g]->R + a.tpb - 1) / a.tpb;
+  }
+  a.nrb = rb;
+  a.N = G == 1 ? w[0]->N : rb * 128;
   a.M = M;
-  a.sx = sx; a.bias = bias; a.y = y; a.ydtype = ydtype; a.ldy = ldy;
+  a.sx = sx; a.ydtype = ydtype;
   a.ws = ws;
   a.P = P;
   char* wsb = static_cast<char*>(ws);
@@ -848,7 +907,7 @@ static cudaError_t launch_tc_impl(const aq_packed* w, const int8_t* xq, const fl
   }
   a.ntb = (M + nt - 1) / nt;
   if (phase == AQ_PHASE_DECODE && P == nullptr) {
-    const DecodePlan p = plan_decode(M, w);
+    const DecodePlan p = plan_tc_decode(M, a.nrb, a.C);
     a.S = p.S;
     if (a.S > kMaxTcSplits) return cudaErrorInvalidValue;  // the split reduction unrolls over kMaxTcSplits
     const size_t cnt_bytes = ((size_t)p.blocks * sizeof(int) + 255) / 256 * 256;
@@ -862,6 +921,20 @@ static cudaError_t launch_tc_impl(const aq_packed* w, const int8_t* xq, const fl
   a.units = a.nrb * a.ntb * a.S;
   const int grid = std::min(a.units, sms);
   const int mode = P ? 2 : (a.S > 1 ? 1 : 0);
+  if (G > 1) {  // grouped launches: decode only (at most 64 tokens)
+    if (phase != AQ_PHASE_DECODE || P != nullptr) return cudaErrorInvalidValue;
+    switch (nt * 4 + mode) {
+#define AQ_TC_CASE_G(NTV)                                                      \
+  case NTV * 4 + 0: return launch_nt<NTV, 0, true>(w, xq, a, grid, st);      \
+  case NTV * 4 + 1: return launch_nt<NTV, 1, true>(w, xq, a, grid, st);
+      AQ_TC_CASE_G(16)
+      AQ_TC_CASE_G(32)
+      AQ_TC_CASE_G(48)
+      AQ_TC_CASE_G(64)
+#undef AQ_TC_CASE_G
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (nt * 4 + mode) {
 #define AQ_TC_CASE(NTV)                                                  \
   case NTV * 4 + 0: return launch_nt<NTV, 0>(w, xq, a, grid, st);      \
@@ -885,12 +958,19 @@ static cudaError_t launch_tc_impl(const aq_packed* w, const int8_t* xq, const fl
 
 cudaError_t launch_tc(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias, void* y,
                       int ydtype, int ldy, void* ws, int32_t* P, int phase, cudaStream_t st) {
-  return launch_tc_impl(w, xq, sx, M, bias, y, ydtype, ldy, ws, P, phase, kWaitTimeoutNs, -1, st);
+  return launch_tc_impl(&w, 1, &bias, &y, &ldy, xq, sx, M, ydtype, ws, P, phase, kWaitTimeoutNs, -1, st);
+}
+
+cudaError_t launch_tc_group(const aq_packed* const* w, int G, const float* const* bias, void* const* y,
+                            const int* ldy, const int8_t* xq, const float* sx, int M, int ydtype, void* ws, int phase,
+                            cudaStream_t st) {
+  return launch_tc_impl(w, G, bias, y, ldy, xq, sx, M, ydtype, ws, nullptr, phase, kWaitTimeoutNs, -1, st);
 }
 
 cudaError_t launch_tc_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, void* y, int ldy,
                               void* ws, int phase, unsigned long long wait_ns, int stop_after, cudaStream_t st) {
-  return launch_tc_impl(w, xq, sx, M, nullptr, y, AQ_F32, ldy, ws, nullptr, phase, wait_ns, stop_after, st);
+  void* yy = y;
+  return launch_tc_impl(&w, 1, nullptr, &yy, &ldy, xq, sx, M, AQ_F32, ws, nullptr, phase, wait_ns, stop_after, st);
 }
 
 }  // namespace aq
