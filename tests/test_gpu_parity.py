@@ -302,6 +302,31 @@ def test_group_decode_matches_separate_calls_and_oracle(M, members):
     assert rc == 0
 
 
+@pytest.mark.parametrize("M,K,bN", [(16, 4096, 128), (40, 8192, 128), (24, 4096, 64), (64, 2048, 64)])
+def test_group_tensor_core_launch(M, K, bN):
+    """A decode group on the tensor cores runs as one launch over the members'
+    concatenated 128-row blocks (split-K partial sums included where the plan
+    splits): bf16 outputs into strided buffers with bias, identical to separate
+    calls (same split plan per member here) and within tolerance of the oracle."""
+    shapes = [(384, K), (256, K), (128, K)]
+    ps, ws, x = _group_case(shapes, M, 1300 + M + K, aq.AQ_PHASE_DECODE, bN=bN, frac8=0.3)
+    xd = dev_bf16(x)
+    grp = aq.Group(ws, aq.AQ_PHASE_DECODE, M)
+    outs_full = [torch.full((M, N + 16), 3.0, device="cuda", dtype=torch.bfloat16) for N, _ in shapes]
+    outs = [o[:, :N] for o, (N, _) in zip(outs_full, shapes)]
+    biases = [torch.linspace(-1, 1, N, device="cuda") for N, _ in shapes]
+    grp(xd, outs, bias=biases)
+    xq, sx = aq.aq_quant_act(xd)
+    for g, (p, w) in enumerate(zip(ps, ws)):
+        sep = aq.aq_linear_decode(w, xq, sx, bias=biases[g], out_dtype=torch.bfloat16)
+        assert torch.equal(outs[g], sep), g
+        assert_output_close(outs[g], oracle_linear(p, x, bias=biases[g].cpu().numpy()))
+        assert (outs_full[g][:, shapes[g][0]:] == 3.0).all()
+    aq.check_all_workspaces()
+    rc, _ = aq.aq_workspace_status(grp.ws)
+    assert rc == 0
+
+
 @pytest.mark.parametrize("M", [1, 300])
 def test_group_prefill_matches_oracle(M):
     shapes = [(512, 768), (384, 768)]
