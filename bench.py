@@ -305,9 +305,15 @@ class Model:
             need = max(aq.aq_expanded_bytes(w) for layer in self.weights for w in layer.values())
             self.tmp = torch.empty(need + 256, dtype=torch.uint8, device=self.dev)
         # groups run as one fused launch (activation preparation inside) up to 2 tokens; from
-        # 3 tokens on as one preparation launch plus one grouped CUDA-core launch (up to 4 tokens,
-        # or up to 8 for groups of three or more) or one tensor-core launch per member
+        # 3 tokens on as one preparation launch plus one linear launch over all members (CUDA
+        # cores up to 4 tokens; tensor cores in decode when every member's rows are whole
+        # 128-row blocks; CUDA cores up to 8 tokens for groups of three or more otherwise), else
+        # one linear launch per member (prefill)
         self.fused = self.phase == aq.AQ_PHASE_DECODE and M <= 2
+        decode = self.phase == aq.AQ_PHASE_DECODE
+        self.one_launch = {kind: len(names) == 1 or (decode and (
+            M <= 4 or all(self.out_dims[nm] % 128 == 0 for nm in names) or (len(names) >= 3 and M <= 8)))
+            for kind, names in self.members.items()}
 
     def step(self, mode="group", chunks=1):
         """Enqueue one pass over every layer (`chunks` passes for a chunked
@@ -325,8 +331,7 @@ class Model:
                 names = self.members[kind]
                 if mode == "group":
                     self.groups[l][kind](self.x[l][kind], [self.y[nm] for nm in names], ws=self.ws)
-                    rows = self.phase == aq.AQ_PHASE_DECODE and (self.M <= 4 or (len(names) >= 3 and self.M <= 8))
-                    n += 1 if self.fused else 1 + (1 if rows else len(names))  # fused, or quantize + members
+                    n += 1 if self.fused else 1 + (1 if self.one_launch[kind] else len(names))  # quantize + linear
                 elif mode == "expanded":
                     for nm in names:
                         aq.aq_linear_prefill_expanded(self.weights[l][nm], self.xq[kind], self.sx[kind],

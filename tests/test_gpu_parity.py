@@ -290,14 +290,27 @@ def test_group_decode_matches_separate_calls_and_oracle(M, members):
     xq, sx = aq.aq_quant_act(xd)
     for g, (p, w) in enumerate(zip(ps, ws)):
         sep = aq.aq_linear_decode(w, xq, sx, bias=biases[g])
-        # a group of three or more runs as one CUDA-core launch up to 8 tokens, where a
-        # single call from 5 tokens on takes the tensor cores: same products, different
-        # FP32 summation order, so only the oracle comparison applies there
-        if not (members >= 3 and 5 <= M <= 8):
-            assert torch.equal(outs[g], sep), g
+        # same kernel family and split plan as the separate call (whole 128-row blocks per member)
+        assert torch.equal(outs[g], sep), g
         assert_output_close(outs[g], oracle_linear(p, x, bias=biases[g].cpu().numpy()))
         assert_output_close(sep, oracle_linear(p, x, bias=biases[g].cpu().numpy()))
     aq.check_all_workspaces()
+    rc, _ = aq.aq_workspace_status(grp.ws)
+    assert rc == 0
+
+
+@pytest.mark.parametrize("M", [5, 8])
+def test_group_rows_launch_for_ragged_members(M):
+    """Three members whose rows are not whole 128-row blocks (64-row tiles, odd
+    tile-row counts) cannot share a tensor-core launch; up to 8 tokens they run as
+    one CUDA-core launch over the codes."""
+    shapes = [(320, 1024), (192, 1024), (64, 1024)]
+    ps, ws, x = _group_case(shapes, M, 1200 + M, aq.AQ_PHASE_DECODE, bN=64, frac8=0.3)
+    grp = aq.Group(ws, aq.AQ_PHASE_DECODE, M)
+    outs = [torch.empty((M, N), device="cuda") for N, _ in shapes]
+    grp(dev_bf16(x), outs)
+    for p, o in zip(ps, outs):
+        assert_output_close(o, oracle_linear(p, x))
     rc, _ = aq.aq_workspace_status(grp.ws)
     assert rc == 0
 

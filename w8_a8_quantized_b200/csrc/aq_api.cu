@@ -361,8 +361,10 @@ static size_t group_ws_bytes(int phase, int M, const aq_packed* const* w, int G)
 
 // A decode group runs as one CUDA-core launch over all members' rows when every
 // member would use the CUDA-core kernel alone, or, up to kRowsMaxM tokens,
-// when it has three or more members (one launch beats one tensor-core launch
-// per member there: q/k/v at 8 tokens, 24.8 against 27.6 us per layer).
+// when it has three or more members and cannot take the grouped tensor-core
+// launch (one CUDA-core launch beats one tensor-core launch per member: q/k/v
+// at 8 tokens, 24.8 against 27.6 us per layer; the grouped tensor-core launch
+// beats both: whole 3B- / 8B- / 14B-class steps at 8 tokens 14-16% faster).
 static bool group_rows(int phase, const aq_packed* const* w, int G, int M) {
   if (phase != AQ_PHASE_DECODE) return false;
   bool all_rows = true, all_supported = true;
@@ -410,7 +412,7 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   int8_t* xq = reinterpret_cast<int8_t*>(base + align256(lin));
   float* sx = reinterpret_cast<float*>(base + align256(lin) + align256((size_t)M * K));
   e = launch_quant_act(x, M, K, ldx, xq, sx, st);
-  if (e == cudaSuccess && group_rows(phase, w, G, M)) {  // one CUDA-core launch over all members' rows
+  if (e == cudaSuccess && group_rows(phase, w, G, M) && !group_tc(phase, w, G, M)) {  // one CUDA-core launch
     DecodeProj d[kMaxGroup];
     for (int g = 0; g < G; ++g) d[g] = decode_proj(w[g], bias ? bias[g] : nullptr, y[g], ldy[g]);
     e = launch_decode_cc(d, G, K, nullptr, 0, xq, sx, M, ydtype, nullptr, ws, st);
