@@ -401,7 +401,9 @@ size_t aq_group_workspace_bytes(int phase, int M, const aq_packed* const* w, int
  *  - Allocates nothing and calls no allocating routine.
  *  - The first call on a device resolves the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture on the device.
+ *    before any stream capture on the device.  The address is kept for the
+ *    process: after a cudaDeviceReset of that device it is stale, and this
+ *    entry must not be called on that device again.
  *  - Each call clears the parts of the array that must start at zero (status
  *    word, split-K counters) on `stream` before launching.
  *  - All calls share the one array: calls that overlap on the GPU (different
