@@ -67,14 +67,14 @@ WORKLOADS = {
 # from an ncu capture of the named workload, valid only while the kernel source is unchanged
 # (sha256 prefix of the source files).
 MEASURED_TRAFFIC = {
-    # four Llama-3.2-3B layers at 1 token (16 launches of the streaming kernel) read 259,320,832 B
-    # and wrote 0 B -> 16,207,552 B per launch (algorithmic: 16,128,638 B per launch)
+    # four Llama-3.2-3B layers at 1 token (16 launches of the streaming kernel) read 259,310,848 B
+    # and wrote 0 B -> 16,206,928 B per launch (algorithmic: 16,128,638 B per launch)
     "decode": {"src": ("w8_a8_quantized_b200/csrc/decode_stream.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
-               "sha": "424e9cf085457b0e", "bytes_per_launch": 16207552},
-    # the Qwen3-4B-shaped prefill's gate projection (N 9728, K 2560, 2048 tokens): 23,162,368 B read,
-    # 28,191,744 B written (the rest of the 79.7 MB fp32 output still in L2 at the end of the launch)
+               "sha": "93bb17d4f34e1fc8", "bytes_per_launch": 16206928},
+    # the Qwen3-4B-shaped prefill's gate projection (N 9728, K 2560, 2048 tokens): 23,168,512 B read,
+    # 26,489,344 B written (the rest of the 79.7 MB fp32 output still in L2 at the end of the launch)
     "prefill": {"src": ("w8_a8_quantized_b200/csrc/tc_linear.cu", "w8_a8_quantized_b200/csrc/aq_internal.cuh"),
-                "sha": "e9795177b774b80c", "bytes_per_launch": 51354112},
+                "sha": "ed409c05043d3c62", "bytes_per_launch": 49657856},
 }
 
 
