@@ -306,13 +306,13 @@ class Model:
             self.tmp = torch.empty(need + 256, dtype=torch.uint8, device=self.dev)
         # groups run as one fused launch (activation preparation inside) up to 2 tokens; from
         # 3 tokens on as one preparation launch plus one linear launch over all members (CUDA
-        # cores up to 4 tokens; tensor cores in decode when every member's rows are whole
+        # cores up to 3 tokens; tensor cores in decode when every member's rows are whole
         # 128-row blocks; CUDA cores up to 8 tokens for groups of three or more otherwise), else
         # one linear launch per member (prefill)
         self.fused = self.phase == aq.AQ_PHASE_DECODE and M <= 2
         decode = self.phase == aq.AQ_PHASE_DECODE
         self.one_launch = {kind: len(names) == 1 or (decode and (
-            M <= 4 or all(self.out_dims[nm] % 128 == 0 for nm in names) or (len(names) >= 3 and M <= 8)))
+            M <= 3 or all(self.out_dims[nm] % 128 == 0 for nm in names) or (len(names) >= 3 and M <= 8)))
             for kind, names in self.members.items()}
 
     def step(self, mode="group", chunks=1):

@@ -137,18 +137,19 @@ def test_host_validation_rejects_before_any_launch():
 
 
 def test_decode_workspace_sizes():
-    """Up to 4 tokens the CUDA-core kernel needs only the status header; above,
+    """Up to 3 tokens the CUDA-core kernel needs only the status header; above,
     the tensor-core split-K partial sums grow with the token count."""
     L = aq.lib()
     s = aq.AqPackedStruct(N=1024, K=3072, bN=128, bK=128, R=8, C=24, T4=100, T8=92,
                           bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
     b1 = L.aq_workspace_bytes(0, 1, ctypes.byref(s))
+    b3 = L.aq_workspace_bytes(0, 3, ctypes.byref(s))
     b4 = L.aq_workspace_bytes(0, 4, ctypes.byref(s))
     b8 = L.aq_workspace_bytes(0, 8, ctypes.byref(s))
     b16 = L.aq_workspace_bytes(0, 16, ctypes.byref(s))
     b32 = L.aq_workspace_bytes(0, 32, ctypes.byref(s))
-    assert b1 == b4 == 256
-    assert b32 > b16 > b8 > 256
+    assert b1 == b3 == 256
+    assert b32 > b16 > b8 > b4 > 256
 
 
 def test_group_workspace_sizes():
