@@ -274,3 +274,48 @@ def test_paper_exact_mode_validation():
     assert q(16, 0, 128, 128, None, 16, 16, None) == -1
     assert q(16, 1, 96, 96, None, 16, 16, None) == -1      # K % 64
     assert q(16, 1, 128, 120, None, 16, 16, None) == -1    # ldx < K
+
+
+def _split_count(M, N, K, sms=148):
+    """Splits of the tensor-core decode plan (a restatement of the rule for this test)."""
+    C, blocks = K // 128, -(-N // 128)
+    per = 5 if M <= 16 else 8 if M <= 32 else 20
+    s = max(1, min(min(C // per, 8), sms // blocks))
+    return 1 if (M >= 32 and 3 * blocks >= sms) else s
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 3072, 3072), (32, 3072, 3072), (64, 3072, 3072), (64, 3072, 8192),
+                                   (32, 8192, 3072), (16, 4096, 14336), (4, 1024, 3072), (64, 4096, 14336)])
+def test_decode_split_plan_in_workspace_sizes(M, N, K):
+    """The workspace of a tensor-core decode call holds the header, one split
+    counter per 128-row block and, with splits, S partial-sum planes of
+    N x (M rounded up to 4) floats: at least 5 / 8 / 20 input tiles per split at
+    <= 16 / <= 32 / <= 64 tokens, one wave, at most 8, and no split from 32
+    tokens when the row blocks fill a third of the GPU."""
+    L = aq.lib()
+    R, C = N // 128, K // 128
+    s = aq.AqPackedStruct(N=N, K=K, bN=128, bK=128, R=R, C=C, T4=R * C, T8=0,
+                          bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    counters = (R * 4 + 255) // 256 * 256
+    S = _split_count(M, N, K)
+    want = 256 + counters + (S * ((M + 3) // 4 * 4) * N * 4 if S > 1 else 0)
+    assert L.aq_workspace_bytes(0, M, ctypes.byref(s)) == want
+
+
+def test_group_workspace_covers_the_grouped_tensor_core_launch():
+    """A decode group whose members are whole 128-row blocks runs as one
+    tensor-core launch over all their rows: its workspace holds that launch's
+    partial sums (split plan over the summed row blocks) before the prepared
+    activations."""
+    L = aq.lib()
+    P = ctypes.POINTER(aq.AqPackedStruct)
+    mk = lambda N: aq.AqPackedStruct(N=N, K=8192, bN=128, bK=128, R=N // 128, C=64, T4=0, T8=(N // 128) * 64,
+                                     bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=16)
+    members = [mk(1024), mk(256), mk(256)]
+    arr = (P * 3)(*[ctypes.pointer(m) for m in members])
+    M, N = 16, 1536
+    S = _split_count(M, N, 8192)
+    blocks = N // 128
+    lin = 256 + (blocks * 4 + 255) // 256 * 256 + S * M * N * 4
+    align = lambda b: (b + 255) // 256 * 256
+    assert L.aq_group_workspace_bytes(0, M, arr, 3) >= align(lin) + align(M * 8192) + align(M * 4)
