@@ -344,7 +344,7 @@ int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int M, int phas
 
 /*
  * Test entry for the failure path of the tensor-core linear kernel (the one that
- * runs prefill and decode from 5 tokens): it runs that kernel with a stage that
+ * runs prefill and decode from 4 tokens): it runs that kernel with a stage that
  * can never fill, without any invalid memory access.  The weight producer stops
  * after `stop_after` input tiles, so the MMA issuer's wait for the next stage,
  * and then every other role's wait, runs out; every bounded wait gives up after

@@ -75,7 +75,7 @@ static constexpr int kMaxSplits = 8;
 static int min_split_tiles(int M) { return M <= 16 ? 5 : M <= 32 ? 8 : 20; }
 
 // Fusing the activation preparation into every CTA of the CUDA-core decode
-// kernel pays off for 1-2 tokens; from 4 tokens on, one preparation kernel plus
+// kernel pays off for 1-2 tokens; from 3 tokens on, one preparation kernel plus
 // a single grouped launch over pre-quantized codes is faster (the per-CTA
 // preparation grows with M).  The fused codes live in shared memory.
 bool rows_fusable(int M, int K) { return M <= 2 && 2 * (size_t)M * K + 16 * (size_t)M <= kFusedMaxBytes; }
