@@ -286,7 +286,8 @@ int aq_paper_quant_act(const uint16_t* x, int M, int K, int ldx, const float* v,
  * Any M >= 1 (the CUDA cores compute it; it is the numerics reference of the
  * paper's own construction, not the per-token layer's fast path).
  * Asynchronous, no workspace.  Errors: AQ_ERR_ARG (null pointer, M < 1,
- * ldy < N, a packed struct of the other scale kind), AQ_ERR_SHAPE, AQ_ERR_CUDA.
+ * M > 1,048,560 (65,535 row groups), ldy < N, a packed struct of the other
+ * scale kind), AQ_ERR_SHAPE, AQ_ERR_CUDA.
  */
 int aq_paper_linear(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* u, const float* bias,
                     float* y, int ldy, void* stream);

@@ -259,6 +259,7 @@ def test_paper_exact_mode_validation():
                                 scale_kind=aq.AQ_SCALES_TILE_FP32, **bufs)
     assert lin(ctypes.byref(bad_geo), 16, 16, 1, None, None, 16, 128, None) == -2
     assert lin(ctypes.byref(paper), 16, 16, 0, None, None, 16, 128, None) == -1      # M < 1
+    assert lin(ctypes.byref(paper), 16, 16, 65536 * 16, None, None, 16, 128, None) == -1  # > 65535 row groups
     assert lin(ctypes.byref(paper), 16, 16, 1, None, None, None, 128, None) == -1    # no output
     assert lin(ctypes.byref(paper), 16, 16, 1, None, None, 16, 100, None) == -1      # ldy < N
     assert lin(ctypes.byref(paper), 24, 16, 1, None, None, 16, 128, None) == -1      # xq not 16-byte aligned

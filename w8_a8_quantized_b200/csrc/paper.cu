@@ -260,6 +260,7 @@ int paper_call(const aq_packed* w, const int8_t* xq, const float* sx, int M, con
   if (!xq || ((uintptr_t)xq & 15) || M < 1 || M > (1 << 20)) return AQ_ERR_ARG;
   if (P == nullptr && (!sx || !y || ldy < w->N)) return AQ_ERR_ARG;
   const int bM = act_group_rows(M), Mp = (M + bM - 1) / bM * bM;
+  if (Mp / bM > 65535) return AQ_ERR_ARG;  // one grid row per activation row group
   PArgs a{w->bitmap, w->tile_idx, w->w4, w->w8, reinterpret_cast<const float*>(w->scales), xq, sx, u, bias, y, P,
           w->N, w->K, w->C, M, bM, ldy};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
