@@ -261,14 +261,14 @@ int aq_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, fl
  *   per group A of 64 features x b_M rows of X~ (rows zero-padded to M'):
  *   s = max(max(0, max A) / 127, max(0, -min A) / 128, 1e-12)
  *   xq = clamp(rint(x~ / s), -128, 127) (fp64 quotient)     sx = (float)s
- *  x   bf16 [M][ldx] (bits as uint16)
- *  v   fp32 [K/64][64][64], V_c[i][k] at (c*64 + i)*64 + k; NULL = identity
+ *  x   bf16 [M][ldx] (bits as uint16), 2-byte aligned
+ *  v   fp32 [K/64][64][64], V_c[i][k] at (c*64 + i)*64 + k, 16-byte aligned; NULL = identity
  *      (then the result equals aq_quant_act_groups).  The sums are formed in
  *      fp64; with the paper's transform seeds (entries 0, +-1, +-1/8) and
  *      bf16 inputs they are exact, so the codes do not depend on the order.
- *  xq  int8 [M'][K], sx fp32 [M'/b_M][K/64], M' = ceil(M / b_M) * b_M.
- * Asynchronous.  Errors: AQ_ERR_ARG (null x / xq / sx, M < 1, K < 64,
- * K % 64, ldx < K), AQ_ERR_CUDA.
+ *  xq  int8 [M'][K], sx fp32 [M'/b_M][K/64] (4-byte aligned), M' = ceil(M / b_M) * b_M.
+ * Asynchronous.  Errors: AQ_ERR_ARG (null x / xq / sx, misaligned x / v / sx,
+ * M < 1, K < 64, K % 64, ldx < K), AQ_ERR_CUDA.
  */
 int aq_paper_quant_act(const uint16_t* x, int M, int K, int ldx, const float* v, int8_t* xq, float* sx,
                        void* stream);
@@ -279,22 +279,24 @@ int aq_paper_quant_act(const uint16_t* x, int M, int K, int ldx, const float* v,
  *   P[m][n][j] = sum_{k in tile column j} xq[m][k] * q[n][k]       (exact INT32)
  *   y[m][r*bN + c] = sum_{i < bN} y~[m][r*bN + i] * U_r[i][c]  (+ bias[r*bN + c])
  *  w     a projection packed by aq_pack_tiles (bK == 64, per-tile fp32 scales)
- *  xq    int8 [M'][K] and sx fp32 [M'/b_M][K/64] as aq_paper_quant_act writes them
+ *  xq    int8 [M'][K] (16-byte aligned) and sx fp32 [M'/b_M][K/64] as aq_paper_quant_act
+ *        writes them; every fp32 pointer here (sx, u, bias, y) 4-byte aligned
  *  u     fp32 [R][bN][bN], U_r[i][c] at (r*bN + i)*bN + c; NULL = identity
  *  bias  fp32 [N] or NULL
  *  y     fp32 [M][ldy]; rows m < M are written, nothing else
  * Any M >= 1 (the CUDA cores compute it; it is the numerics reference of the
  * paper's own construction, not the per-token layer's fast path).
- * Asynchronous, no workspace.  Errors: AQ_ERR_ARG (null pointer, M < 1,
- * M > 1,048,560 (65,535 row groups), ldy < N, a packed struct of the other
- * scale kind), AQ_ERR_SHAPE, AQ_ERR_CUDA.
+ * Asynchronous, no workspace.  Errors: AQ_ERR_ARG (null or misaligned pointer,
+ * M < 1, M > 1,048,560 (65,535 row groups), ldy < N, a packed struct of the
+ * other scale kind), AQ_ERR_SHAPE, AQ_ERR_CUDA.
  */
 int aq_paper_linear(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* u, const float* bias,
                     float* y, int ldy, void* stream);
 
 /*
  * Test entry: the exact integer tile products P[m][n][j] (int32 [M][N][K/64])
- * of aq_paper_linear, as its kernel forms them.  Errors as aq_paper_linear.
+ * of aq_paper_linear, as its kernel forms them (P 4-byte aligned).  Errors as
+ * aq_paper_linear.
  */
 int aq_debug_paper_partials(const aq_packed* w, const int8_t* xq, int M, int32_t* P, void* stream);
 

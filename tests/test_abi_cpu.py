@@ -263,7 +263,12 @@ def test_paper_exact_mode_validation():
     assert lin(ctypes.byref(paper), 16, 16, 1, None, None, None, 128, None) == -1    # no output
     assert lin(ctypes.byref(paper), 16, 16, 1, None, None, 16, 100, None) == -1      # ldy < N
     assert lin(ctypes.byref(paper), 24, 16, 1, None, None, 16, 128, None) == -1      # xq not 16-byte aligned
+    assert lin(ctypes.byref(paper), 16, 18, 1, None, None, 16, 128, None) == -1      # sx not 4-byte aligned
+    assert lin(ctypes.byref(paper), 16, 16, 1, 18, None, 16, 128, None) == -1        # u
+    assert lin(ctypes.byref(paper), 16, 16, 1, None, 18, 16, 128, None) == -1        # bias
+    assert lin(ctypes.byref(paper), 16, 16, 1, None, None, 18, 128, None) == -1      # y
     assert L.aq_debug_paper_partials(ctypes.byref(paper), 16, 1, None, None) == -1
+    assert L.aq_debug_paper_partials(ctypes.byref(paper), 16, 1, 18, None) == -1    # P not 4-byte aligned
     # the per-token layer refuses a paper-form struct
     paper128 = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
                                  scale_kind=aq.AQ_SCALES_TILE_FP32, **bufs)
@@ -275,6 +280,9 @@ def test_paper_exact_mode_validation():
     assert q(16, 0, 128, 128, None, 16, 16, None) == -1
     assert q(16, 1, 96, 96, None, 16, 16, None) == -1      # K % 64
     assert q(16, 1, 128, 120, None, 16, 16, None) == -1    # ldx < K
+    assert q(16, 1, 128, 128, 24, 16, 16, None) == -1      # V staged with 16-byte loads
+    assert q(17, 1, 128, 128, None, 16, 16, None) == -1    # x read as 2-byte words
+    assert q(16, 1, 128, 128, None, 16, 18, None) == -1    # sx written as 4-byte words
 
 
 def _split_count(M, N, K, sms=148):

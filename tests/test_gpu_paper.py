@@ -109,3 +109,21 @@ def test_paper_linear_without_transforms_and_with_search():
     xq, sx = aq.aq_paper_quant_act(dev_bf16(x_bits))
     y = aq.aq_paper_linear(packed, xq, sx, M)
     assert_output_close(y, ref["y"])
+
+
+def test_paper_operands_are_checked_before_any_launch():
+    """Codes, scales and token counts that do not match the packed weights raise
+    on the host: the kernels read xq as [M'][K] and sx as [M'/b_M][K/64]."""
+    _, packed, x_bits, v_blocks, _, _ = _paper_case(5, 256, 576, 64, 0.4, 2500)
+    xq, sx = aq.aq_paper_quant_act(dev_bf16(x_bits), _dev_f32(np.stack(v_blocks)))
+    assert xq.shape == (16, 576) and sx.shape == (1, 9)
+    with pytest.raises(ValueError):
+        aq.aq_paper_linear(packed, xq[:, :512].contiguous(), sx, 5)   # K does not match the weights
+    with pytest.raises(ValueError):
+        aq.aq_paper_linear(packed, xq, sx, 17)                        # 17 tokens pad to 32 code rows
+    with pytest.raises(ValueError):
+        aq.aq_paper_linear(packed, xq, sx[:, :4].contiguous(), 5)     # fewer group scales than tiles
+    with pytest.raises(ValueError):
+        aq.aq_paper_linear(packed, xq, sx, 0)
+    with pytest.raises(ValueError):
+        aq.aq_debug_paper_partials(packed, xq, 17)

@@ -240,14 +240,32 @@ def aq_paper_quant_act(x: torch.Tensor, v: torch.Tensor = None):
     return xq, sx
 
 
+def _paper_operands(w: PackedWeights, xq: torch.Tensor, M: int) -> int:
+    """Check the paper-exact layer's codes against the packed weights: the kernel
+    reads xq as [M'][K] (M' = M rounded up to whole row groups); returns the
+    number of activation row groups M' / b_M."""
+    if w.struct.scale_kind != AQ_SCALES_TILE_FP32:
+        raise ValueError("w must be packed by aq_pack_tiles (per-tile fp32 scales)")
+    _need(xq, "xq", torch.int8, w.device)
+    bM = int(lib().aq_act_group_rows(M)) if M >= 1 else 0
+    if bM == 0:
+        raise ValueError("M must be at least 1")
+    Mp = -(-M // bM) * bM
+    if xq.dim() != 2 or xq.shape[1] != w.K or xq.shape[0] < Mp:
+        raise ValueError(f"xq must be [>= {Mp}][{w.K}] (M = {M} padded to whole row groups), got {tuple(xq.shape)}")
+    return Mp // bM
+
+
 def aq_paper_linear(w: PackedWeights, xq: torch.Tensor, sx: torch.Tensor, M: int, u: torch.Tensor = None,
                     bias: torch.Tensor = None, out: torch.Tensor = None) -> torch.Tensor:
     """Paper-exact layer (eq. 19, then Y = Y~ U): w from aq_pack_tiles, (xq, sx)
     from aq_paper_quant_act, u float32 [R][bN][bN] (None = identity), bias
     float32 [N] -> y float32 [M][N]."""
     dev = w.device
-    _need(xq, "xq", torch.int8, dev)
+    groups = _paper_operands(w, xq, M)
     _need(sx, "sx", torch.float32, dev)
+    if sx.numel() < groups * w.C:
+        raise ValueError(f"sx must hold [{groups}][{w.C}] group scales, got {sx.numel()} values")
     if u is not None:
         _need(u, "u", torch.float32, dev)
         if tuple(u.shape) != (w.R, w.bN, w.bN):
@@ -272,7 +290,7 @@ def aq_paper_linear(w: PackedWeights, xq: torch.Tensor, sx: torch.Tensor, M: int
 def aq_debug_paper_partials(w: PackedWeights, xq: torch.Tensor, M: int) -> torch.Tensor:
     """Exact integer tile products of the paper-exact layer: int32 [M][N][K/64]."""
     dev = w.device
-    _need(xq, "xq", torch.int8, dev)
+    _paper_operands(w, xq, M)
     P = torch.zeros((M, w.N, w.C), dtype=torch.int32, device=dev)
     with torch.cuda.device(dev):
         _check(lib().aq_debug_paper_partials(ctypes.byref(w.struct), xq.data_ptr(), M, P.data_ptr(), _stream(dev)),

@@ -259,6 +259,8 @@ int paper_call(const aq_packed* w, const int8_t* xq, const float* sx, int M, con
   if (rc != AQ_OK) return rc;
   if (!xq || ((uintptr_t)xq & 15) || M < 1 || M > (1 << 20)) return AQ_ERR_ARG;
   if (P == nullptr && (!sx || !y || ldy < w->N)) return AQ_ERR_ARG;
+  // fp32 / int32 operands are read and written as 4-byte words
+  if (((uintptr_t)sx | (uintptr_t)u | (uintptr_t)bias | (uintptr_t)y | (uintptr_t)P) & 3) return AQ_ERR_ARG;
   const int bM = act_group_rows(M), Mp = (M + bM - 1) / bM * bM;
   if (Mp / bM > 65535) return AQ_ERR_ARG;  // one grid row per activation row group
   PArgs a{w->bitmap, w->tile_idx, w->w4, w->w8, reinterpret_cast<const float*>(w->scales), xq, sx, u, bias, y, P,
@@ -277,6 +279,8 @@ extern "C" int aq_paper_quant_act(const uint16_t* x, int M, int K, int ldx, cons
                                   void* stream) {
   if (!x || !xq || !sx || M < 1 || M > (1 << 20) || K < kGroup || K % kGroup || K > (1 << 20) || ldx < K)
     return AQ_ERR_ARG;
+  // V is staged with 16-byte loads; x is read as 2-byte words, sx written as 4-byte words
+  if (((uintptr_t)v & 15) || ((uintptr_t)x & 1) || ((uintptr_t)sx & 3)) return AQ_ERR_ARG;
   const int bM = act_group_rows(M), Mp = (M + bM - 1) / bM * bM;
   const long long blocks = (long long)(Mp / bM) * (K / kGroup);
   if (blocks > 0x7fffffffll) return AQ_ERR_ARG;
