@@ -314,13 +314,16 @@ size_t aq_workspace_bytes(int phase, int M, const aq_packed* w);
  * App. E.3 eq. 19 and the ordered split reduction after it).
  *  w     host struct describing device buffers produced by aq_pack
  *  xq    int8 [M][K] device, 16-byte aligned (from aq_quant_act)
- *  sx    fp32 [M] device
- *  bias  fp32 [N] device or NULL
- *  y     [M][ldy] device, fp32 or bf16 per ydtype (aq_dtype), ldy >= N
- *  ws    device workspace of >= aq_workspace_bytes(AQ_PHASE_DECODE, M, w) bytes
+ *  sx    fp32 [M] device, 4-byte aligned
+ *  bias  fp32 [N] device, 4-byte aligned, or NULL
+ *  y     [M][ldy] device, fp32 or bf16 per ydtype (aq_dtype), aligned to its
+ *        element, ldy >= N
+ *  ws    device workspace of >= aq_workspace_bytes(AQ_PHASE_DECODE, M, w) bytes,
+ *        16-byte aligned
  * Split-K partial sums are reduced in increasing split order, so results are
  * bitwise reproducible for a given (M, w) on a given GPU.
- * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
+ * Errors: AQ_ERR_ARG (also a misaligned pointer), AQ_ERR_SHAPE,
+ * AQ_ERR_WORKSPACE (ws NULL or too small), AQ_ERR_CUDA.
  */
 int aq_linear_decode(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
                      void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream);
@@ -337,7 +340,7 @@ int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const float* sx, int
 
 /*
  * Test entry: the exact per-tile INT32 products P[m][n][j] (eq. 19, the
- * parenthesized product) written to P int32 [M][N][C] device, computed by the
+ * parenthesized product) written to P int32 [M][N][C] device (4-byte aligned), computed by the
  * same data path (tile location, INT4 expansion, integer products) as the
  * linear call of `phase`.  Not a hot-path call.
  * Errors: AQ_ERR_ARG, AQ_ERR_SHAPE, AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
@@ -373,14 +376,19 @@ int aq_debug_linear_stalled(const aq_packed* w, const int8_t* xq, const float* s
  *  phase  AQ_PHASE_DECODE (1 <= M <= 64) or AQ_PHASE_PREFILL (M >= 1)
  *  w      host array of G pointers to packed projections with equal K
  *  x      bf16 [M][ldx] device (bits as uint16), 16-byte aligned, ldx % 8 == 0
- *  bias   host array of G device pointers (each fp32 [N_g] or NULL), or NULL
- *  y      host array of G device outputs [M][ldy[g]], fp32 or bf16 per ydtype
+ *  bias   host array of G device pointers (each fp32 [N_g], 4-byte aligned, or NULL), or NULL
+ *  y      host array of G device outputs [M][ldy[g]], fp32 or bf16 per ydtype, aligned to
+ *         their element
  *  ldy    host array of G leading dimensions, ldy[g] >= N_g
- *  ws     device workspace of >= aq_group_workspace_bytes(phase, M, w, G) bytes
- * Decode with at most 8 tokens runs as ONE launch: every CTA quantizes the
- * input it needs itself (same arithmetic as aq_quant_act) and the members'
- * output rows are concatenated.  Other cases quantize x once into the
- * workspace and run each member on it.
+ *  ws     device workspace of >= aq_group_workspace_bytes(phase, M, w, G) bytes, 16-byte aligned
+ * Decode with one or two tokens runs as ONE launch where the codes fit in
+ * shared memory: every CTA quantizes the input it needs itself (same
+ * arithmetic as aq_quant_act) and the members' output rows are concatenated.
+ * Otherwise x is quantized once into the workspace and the members run on it,
+ * in one launch over all their rows where the decode plan allows it (the
+ * CUDA-core kernel up to 3 tokens, and for three members up to 8 tokens; the
+ * tensor-core kernel from 4 tokens when every member has whole 128-row blocks
+ * and all share one tile height), else in one launch per member.
  * Errors: AQ_ERR_ARG (also G outside 1..3, unequal K), AQ_ERR_SHAPE,
  * AQ_ERR_WORKSPACE, AQ_ERR_CUDA.
  */

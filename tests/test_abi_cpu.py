@@ -113,6 +113,24 @@ def test_host_validation_rejects_before_any_launch():
     assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 64, 16, 1 << 20, None) == -1
     assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, None, 0, None) == -5
     assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, 16, 8, None) == -5
+    # token scales, bias and fp32 outputs are 4-byte words, bf16 outputs 2-byte words, the workspace 16-byte aligned
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 18, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, 18, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 18, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 17, 1, 128, 16, 1 << 20, None) == -1
+    assert L.aq_linear_decode(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, 24, 1 << 20, None) == -1
+    assert L.aq_linear_prefill(ctypes.byref(s), 16, 16, 1, None, 16, 0, 128, 24, 1 << 20, None) == -1
+    assert L.aq_linear_decode_noalloc(ctypes.byref(s), 16, 18, 1, None, 16, 0, 128, None) == -1
+    assert L.aq_linear_decode_noalloc(ctypes.byref(s), 16, 16, 1, None, 17, 1, 128, None) == -1
+    assert L.aq_debug_tile_partials(ctypes.byref(s), 16, 1, 1, 18, 16, 1 << 20, None) == -1
+    ws_args = [ctypes.pointer(s)]
+    members = (ctypes.POINTER(aq.AqPackedStruct) * 1)(*ws_args)
+    ys, lds = (ctypes.c_void_p * 1)(18), (ctypes.c_int * 1)(128)
+    assert L.aq_linear_group(0, members, 1, 16, 128, 1, None, ys, lds, 0, 16, 1 << 20, None) == -1
+    biases = (ctypes.c_void_p * 1)(18)
+    ys[0] = 16
+    assert L.aq_linear_group(0, members, 1, 16, 128, 1, biases, ys, lds, 0, 16, 1 << 20, None) == -1
+    assert L.aq_linear_group(0, members, 1, 16, 128, 1, None, ys, lds, 0, 24, 1 << 20, None) == -1
     # packed buffers moved by bulk copies (w4, w8, scales) must be 16-byte aligned
     mis = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
                             bitmap=16, row_off4=16, row_off8=16, tile_idx=16, w4=16, w8=16, scales=18)

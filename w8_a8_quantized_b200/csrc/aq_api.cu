@@ -187,22 +187,37 @@ extern "C" int aq_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq
                                                                                                    : AQ_ERR_CUDA;
 }
 
-static int check_linear(const aq_packed* w, const int8_t* xq, const float* sx, int M, const void* y, int ydtype,
-                        int ldy) {
+namespace aq {
+// Token scales and bias are fetched as 4-byte words (cp.async of 4 bytes),
+// outputs stored as 4- or 2-byte words: a pointer off that grain is an
+// argument error, not a misaligned access on the GPU.
+bool operands_misaligned(const float* sx, const float* bias, const void* y, int ydtype) {
+  return (((uintptr_t)sx | (uintptr_t)bias) & 3) != 0 || ((uintptr_t)y & (ydtype == AQ_F32 ? 3u : 1u)) != 0;
+}
+}  // namespace aq
+
+static int check_linear(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
+                        const void* y, int ydtype, int ldy) {
   int rc = validate_packed(w);
   if (rc != AQ_OK) return rc;
   if (!xq || !sx || !y || M < 1 || ldy < w->N) return AQ_ERR_ARG;
   if (ydtype != AQ_F32 && ydtype != AQ_BF16) return AQ_ERR_ARG;
-  if ((uintptr_t)xq & 15) return AQ_ERR_ARG;
+  if (((uintptr_t)xq & 15) || operands_misaligned(sx, bias, y, ydtype)) return AQ_ERR_ARG;
   return AQ_OK;
+}
+
+// The workspace holds split-K partial sums written as 16-byte vectors.
+static int check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return AQ_ERR_WORKSPACE;
+  return ((uintptr_t)ws & 15) ? AQ_ERR_ARG : AQ_OK;
 }
 
 extern "C" int aq_linear_decode(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
                                 void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream) {
-  int rc = check_linear(w, xq, sx, M, y, ydtype, ldy);
+  int rc = check_linear(w, xq, sx, M, bias, y, ydtype, ldy);
   if (rc != AQ_OK) return rc;
   if (M > kMaxDecodeM) return AQ_ERR_ARG;
-  if (!ws || ws_bytes < decode_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
+  if ((rc = check_ws(ws, ws_bytes, decode_ws_bytes(M, w))) != AQ_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (plan_decode(M, w).kernel == 0) {
@@ -216,9 +231,9 @@ extern "C" int aq_linear_decode(const aq_packed* w, const int8_t* xq, const floa
 
 extern "C" int aq_linear_prefill(const aq_packed* w, const int8_t* xq, const float* sx, int M, const float* bias,
                                  void* y, int ydtype, int ldy, void* ws, size_t ws_bytes, void* stream) {
-  int rc = check_linear(w, xq, sx, M, y, ydtype, ldy);
+  int rc = check_linear(w, xq, sx, M, bias, y, ydtype, ldy);
   if (rc != AQ_OK) return rc;
-  if (!ws || ws_bytes < prefill_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
+  if ((rc = check_ws(ws, ws_bytes, prefill_ws_bytes(M, w))) != AQ_OK) return rc;
   cudaError_t e = launch_tc(w, xq, sx, M, bias, y, ydtype, ldy, ws, nullptr, AQ_PHASE_PREFILL,
                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? AQ_OK : AQ_ERR_CUDA;
@@ -253,9 +268,9 @@ extern "C" int aq_expand_int8(const aq_packed* w, void* buf, size_t buf_bytes, a
 extern "C" int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, const float* sx, int M,
                                           const float* bias, void* y, int ydtype, int ldy, void* ws, size_t ws_bytes,
                                           void* tmp, size_t tmp_bytes, void* stream) {
-  int rc = check_linear(w, xq, sx, M, y, ydtype, ldy);
+  int rc = check_linear(w, xq, sx, M, bias, y, ydtype, ldy);
   if (rc != AQ_OK) return rc;
-  if (!ws || ws_bytes < prefill_ws_bytes(M, w)) return AQ_ERR_WORKSPACE;
+  if ((rc = check_ws(ws, ws_bytes, prefill_ws_bytes(M, w))) != AQ_OK) return rc;
   if (!tmp || ((uintptr_t)tmp & 255)) return AQ_ERR_ARG;
   if (tmp_bytes < expanded_bytes(w)) return AQ_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -273,7 +288,8 @@ extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int 
   if (!xq || !P || M < 1 || ((uintptr_t)xq & 15)) return AQ_ERR_ARG;
   if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return AQ_ERR_ARG;
   if (phase == AQ_PHASE_DECODE && M > kMaxDecodeM) return AQ_ERR_ARG;
-  if (!ws || ws_bytes < kWsHeader) return AQ_ERR_WORKSPACE;
+  if ((uintptr_t)P & 3) return AQ_ERR_ARG;
+  if ((rc = check_ws(ws, ws_bytes, kWsHeader)) != AQ_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (phase == AQ_PHASE_DECODE && plan_decode(M, w).kernel == 0) {
@@ -287,13 +303,13 @@ extern "C" int aq_debug_tile_partials(const aq_packed* w, const int8_t* xq, int 
 extern "C" int aq_debug_linear_stalled(const aq_packed* w, const int8_t* xq, const float* sx, int M, int phase,
                                        float* y, int ldy, void* ws, size_t ws_bytes, unsigned long long wait_ns,
                                        int stop_after, void* stream) {
-  int rc = check_linear(w, xq, sx, M, y, AQ_F32, ldy);
+  int rc = check_linear(w, xq, sx, M, nullptr, y, AQ_F32, ldy);
   if (rc != AQ_OK) return rc;
   if (phase != AQ_PHASE_DECODE && phase != AQ_PHASE_PREFILL) return AQ_ERR_ARG;
   if (phase == AQ_PHASE_DECODE && (M > kMaxDecodeM || plan_decode(M, w).kernel != 1)) return AQ_ERR_ARG;
   if (wait_ns < 100000ull || wait_ns > 10000000000ull || stop_after < 0) return AQ_ERR_ARG;
   const size_t need = phase == AQ_PHASE_DECODE ? decode_ws_bytes(M, w) : prefill_ws_bytes(M, w);
-  if (!ws || ws_bytes < need) return AQ_ERR_WORKSPACE;
+  if ((rc = check_ws(ws, ws_bytes, need)) != AQ_OK) return rc;
   return launch_tc_stalled(w, xq, sx, M, y, ldy, ws, phase, wait_ns, stop_after, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? AQ_OK
@@ -393,8 +409,9 @@ extern "C" int aq_linear_group(int phase, const aq_packed* const* w, int G, cons
   if (rc != AQ_OK) return rc;
   if (!y || !ldy || (ydtype != AQ_F32 && ydtype != AQ_BF16)) return AQ_ERR_ARG;
   for (int g = 0; g < G; ++g)
-    if (!y[g] || ldy[g] < w[g]->N) return AQ_ERR_ARG;
-  if (!ws || ws_bytes < group_ws_bytes(phase, M, w, G)) return AQ_ERR_WORKSPACE;
+    if (!y[g] || ldy[g] < w[g]->N || operands_misaligned(nullptr, bias ? bias[g] : nullptr, y[g], ydtype))
+      return AQ_ERR_ARG;
+  if ((rc = check_ws(ws, ws_bytes, group_ws_bytes(phase, M, w, G))) != AQ_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int K = w[0]->K;
   cudaError_t e = cudaSuccess;

@@ -20,6 +20,8 @@
 #include "aq_internal.cuh"
 
 namespace aq {
+bool operands_misaligned(const float* sx, const float* bias, const void* y, int ydtype);  // aq_api.cu
+
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB
@@ -55,7 +57,7 @@ extern "C" int aq_linear_decode_noalloc(const aq_packed* w, const int8_t* xq, co
   if (rc != AQ_OK) return rc;
   if (!xq || !sx || !y || M < 1 || M > kMaxDecodeM || ldy < w->N) return AQ_ERR_ARG;
   if (ydtype != AQ_F32 && ydtype != AQ_BF16) return AQ_ERR_ARG;
-  if ((uintptr_t)xq & 15) return AQ_ERR_ARG;
+  if (((uintptr_t)xq & 15) || operands_misaligned(sx, bias, y, ydtype)) return AQ_ERR_ARG;
   const size_t need = decode_ws_bytes(M, w);
   if (need > kNoAllocScratchBytes) return AQ_ERR_WORKSPACE;  // beyond the fixed scratch: use aq_linear_decode
   void* scratch = nullptr;
