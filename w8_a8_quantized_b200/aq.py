@@ -548,9 +548,10 @@ class Group:
             if o.dim() != 2 or o.shape[0] < self.M or o.shape[1] < w.N:
                 raise ValueError(f"each output must be at least [M][N] = [{self.M}][{w.N}]")
         if bias is not None and (len(bias) != G or any(b is not None and (b.dtype != torch.float32 or
-                                                                       b.device != dev or b.numel() < w.N)
+                                                                       b.device != dev or b.numel() < w.N or
+                                                                       not b.is_contiguous())
                                                       for b, w in zip(bias, self.weights))):
-            raise ValueError("bias must hold one float32 [N] tensor (or None) per member")
+            raise ValueError("bias must hold one contiguous float32 [N] tensor (or None) per member")
         dt = outs[0].dtype
         if dt not in (torch.float32, torch.bfloat16) or any(o.dtype != dt or o.device != dev or o.stride(1) != 1
                                                              for o in outs):
