@@ -231,6 +231,21 @@ def _quantize_activation_groups_symmetric(x_tilde):  # groups with the +-127 ran
     return codes, scales, Mp
 
 
+def _weight_tiles_scaled_by_first_row(w_tilde, pmap, bN, bK, search):  # the tile scale from its first row only
+    w = np.asarray(w_tilde, np.float64)
+    N, K = w.shape
+    codes = np.zeros((N, K), np.int8)
+    scales = np.zeros((N // bN, K // bK), np.float32)
+    for r in range(N // bN):
+        for j in range(K // bK):
+            tile = w[r * bN:(r + 1) * bN, j * bK:(j + 1) * bK]
+            b = 4 if int(pmap[r, j]) == ao.W4 else 8
+            s = ao.search_scale(tile[0], b) if search else ao.endpoint_scale(tile[0], b)
+            codes[r * bN:(r + 1) * bN, j * bK:(j + 1) * bK] = ao.quantize_with_scale(tile, s, b)
+            scales[r, j] = np.float32(s)
+    return codes, scales
+
+
 def _reconstruct_groups_first_row_group(xq, sx, qw, sw, bN, bK, M):  # every row scaled by row group 0
     sx0 = np.repeat(np.asarray(sx)[:1], len(sx), axis=0)
     return _REAL_PN["reconstruct_groups"](xq, sx0, qw, sw, bN, bK, M)
@@ -281,6 +296,8 @@ MISTAKES = {
     "packed bytes without the index table": (ao, "packed_bytes", _packed_bytes_no_table),
     "H64 not normalized": (pn, "hadamard64", _hadamard_unnormalized),
     "activation row groups of 8": (pn, "row_group", _row_group_eight),
+    "activation groups of 32 features": (pn, "GROUP", 32),
+    "weight tile scale from its first row": (pn, "quantize_weight_tiles", _weight_tiles_scaled_by_first_row),
     "one token grouped as 16 rows": (pn, "row_group", _row_group_always_sixteen),
     "activation groups with the symmetric range": (pn, "quantize_activation_groups",
                                                     _quantize_activation_groups_symmetric),
