@@ -527,7 +527,7 @@ def oracle_run(wl, budget_s, M):
     """Time the CPU oracle on a bounded sample of the workload: whole projections
     of the first layers (unpack of the packed form, activation quantization,
     integer tile products, fp64 rescale), until `budget_s` seconds are used.
-    Returns (packed bytes done, MACs done, seconds, description)."""
+    Returns (packed bytes done, MACs done, seconds, process CPU seconds, description)."""
     import oracle
     from w8_a8_quantized_b200 import synth
     cfg = CFG_ID[wl["model"]]
@@ -536,16 +536,17 @@ def oracle_run(wl, budget_s, M):
     done_bytes = done_macs = 0
     n_proj = 0
     rows = M if wl["phase"] == "decode" else min(M, 64)
-    t_used = 0.0
+    t_used = cpu_used = 0.0
     for l in range(layers):
         for pid, (name, N, K) in enumerate(projs):
             p = synth.projection_inputs(N, K, wl["bN"], 128, wl["frac8"], (cfg, l, pid))
             pk = oracle.pack(p.codes, p.scales, p.pmap, wl["bN"], 128)
             x = synth.activations(rows, K, (cfg, l, 999, rows), outlier_frac=wl["outlier"])
-            t0 = time.perf_counter()
+            t0, c0 = time.perf_counter(), time.process_time()
             xq, sx = oracle.quant_act(x)
             oracle.linear_packed(pk, xq, sx)
             t_used += time.perf_counter() - t0
+            cpu_used += time.process_time() - c0
             done_bytes += oracle.packed_bytes(pk)
             done_macs += N * K * rows
             n_proj += 1
@@ -555,7 +556,7 @@ def oracle_run(wl, budget_s, M):
             break
     desc = (f"{n_proj} whole projections of the first layer(s) of the workload, {rows} token(s) each, "
             f"unpack + quantize + tile products + fp64 rescale")
-    return done_bytes, done_macs, t_used, desc
+    return done_bytes, done_macs, t_used, cpu_used, desc
 
 
 def cpu_model() -> str:
@@ -569,7 +570,8 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_threads():
+def blas_threads():
+    """Threads of the BLAS pool the oracle's matrix products may use."""
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
@@ -578,22 +580,29 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+def threads_used(cpu_s, wall_s):
+    """Cores the timed region actually kept busy: process CPU time (all threads)
+    over wall time, at least 1."""
+    return max(1.0, round(cpu_s / wall_s, 1)) if wall_s > 0 else 1.0
+
+
 def cpu_baseline(wl, budget_s, decode):
     """The oracle on the host cores, once with one BLAS thread and once with the
-    default thread count (all cores); `value` and `cores` are the all-core run's."""
+    default BLAS pool (all cores offered); `value` and `cores` are the second
+    run's, `cores` being the cores it kept busy (CPU time over wall time)."""
     from threadpoolctl import threadpool_limits
     unit = "GB/s" if decode else "TOPS"
     out = {"kind": "oracle", "unit": unit, "cpu": cpu_model(), "nproc": os.cpu_count()}
     for label in ("single_thread", "all_cores"):
         if label == "single_thread":
             with threadpool_limits(limits=1, user_api="blas"):
-                b, macs, t, desc = oracle_run(wl, budget_s, wl["M"])
-            threads = 1
+                b, macs, t, c, desc = oracle_run(wl, budget_s, wl["M"])
+            pool = 1
         else:
-            b, macs, t, desc = oracle_run(wl, budget_s, wl["M"])
-            threads = cpu_threads()
-        out[label] = {"value": b / t / 1e9 if decode else 2.0 * macs / t / 1e12, "threads": threads,
-                      "sample": desc}
+            b, macs, t, c, desc = oracle_run(wl, budget_s, wl["M"])
+            pool = blas_threads()
+        out[label] = {"value": b / t / 1e9 if decode else 2.0 * macs / t / 1e12, "blas_threads": pool,
+                      "threads": threads_used(c, t), "sample": desc}
     out["value"] = out["all_cores"]["value"]
     out["cores"] = out["all_cores"]["threads"]
     out["sample"] = out["all_cores"]["sample"]
@@ -723,15 +732,16 @@ def run_reference(args, wl, peaks):
         prepared.append((oracle.pack(p.codes, p.scales, p.pmap, wl["bN"], 128),
                          synth.activations(rows, K, (cfg, 0, 999, rows), outlier_frac=wl["outlier"]), N * K))
     tot_b = tot_macs = 0
-    tot_t = 0.0
+    tot_t = tot_c = 0.0
     for i in range(args.warmup + args.steps):
         pk, x, nk = prepared[i % len(prepared)]
-        t0 = time.perf_counter()
+        t0, c0 = time.perf_counter(), time.process_time()
         xq, sx = oracle.quant_act(x)
         oracle.linear_packed(pk, xq, sx)
-        dt = time.perf_counter() - t0
+        dt, dc = time.perf_counter() - t0, time.process_time() - c0
         if i >= args.warmup:
             tot_t += dt
+            tot_c += dc
             tot_b += oracle.packed_bytes(pk)
             tot_macs += nk * rows
     decode = wl["phase"] == "decode"
@@ -744,7 +754,8 @@ def run_reference(args, wl, peaks):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "model_shape": wl["model"], "phase": wl["phase"],
                        "tokens": rows},
-            "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(), "nproc": os.cpu_count(),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads_used(tot_c, tot_t),
+                             "blas_threads": blas_threads(), "nproc": os.cpu_count(),
                              "cpu": cpu_model(), "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
