@@ -586,14 +586,14 @@ def threads_used(cpu_s, wall_s):
     return max(1.0, round(cpu_s / wall_s, 1)) if wall_s > 0 else 1.0
 
 
-def cpu_baseline(wl, budget_s, decode):
+def cpu_baseline(wl, budget_s, decode, legs=("single_thread", "all_cores")):
     """The oracle on the host cores, once with one BLAS thread and once with the
     default BLAS pool (all cores offered); `value` and `cores` are the second
     run's, `cores` being the cores it kept busy (CPU time over wall time)."""
     from threadpoolctl import threadpool_limits
     unit = "GB/s" if decode else "TOPS"
     out = {"kind": "oracle", "unit": unit, "cpu": cpu_model(), "nproc": os.cpu_count()}
-    for label in ("single_thread", "all_cores"):
+    for label in legs:
         if label == "single_thread":
             with threadpool_limits(limits=1, user_api="blas"):
                 b, macs, t, c, desc = oracle_run(wl, budget_s, wl["M"])
@@ -709,6 +709,11 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, 6.0, decode)
+        for label, wname, over, *_ in by_workload_plan(args.steps, args.warmup):
+            if label in line.get("by_workload", {}):  # a shorter sample, all cores only
+                wl2 = dict(WORKLOADS[wname], **over)
+                line["by_workload"][label]["cpu_baseline"] = cpu_baseline(wl2, 1.0, wl2["phase"] == "decode",
+                                                                          legs=("all_cores",))
 
     if dist_on:
         torch.distributed.barrier()
