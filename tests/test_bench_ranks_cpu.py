@@ -54,3 +54,17 @@ def test_replicas_report_slowest_rank_and_whole_job_rate(world):
 def test_job_rate_single_rank():
     import bench
     assert bench.job_rate(1, 2e12, 10.0, 1e12) == pytest.approx(200.0)
+
+
+def test_cpu_baseline_reports_rate_and_measured_cores():
+    """The CPU-baseline leg on the smallest workload with a tiny budget: both legs
+    present, rates positive, `cores` measured (at least 1, at most the host's)."""
+    import bench
+    wl = dict(bench.WORKLOADS["decode-single-2048"])
+    out = bench.cpu_baseline(wl, 0.05, True)
+    assert out["kind"] == "oracle" and out["unit"] == "GB/s"
+    assert out["single_thread"]["blas_threads"] == 1 and out["single_thread"]["value"] > 0
+    assert out["value"] == out["all_cores"]["value"] > 0
+    assert 1.0 <= out["cores"] <= (os.cpu_count() or 1) + 0.5
+    short = bench.cpu_baseline(wl, 0.05, True, legs=("all_cores",))
+    assert "single_thread" not in short and short["value"] > 0
