@@ -33,6 +33,29 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(L, name), name
 
 
+def test_binding_argument_counts_match_the_header():
+    """Every declaration's parameter count equals the length of the binding's
+    ctypes argtypes for it (a missing or extra argument would be marshalled
+    silently)."""
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "aq.h")).read(), flags=re.S)
+    decls = dict(re.findall(r"\b(aq_\w+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S))
+    assert set(decls) == set(_declared_functions())
+    L = aq.lib()
+    c_scalars = {"int": (ctypes.c_int, False), "size_t": (ctypes.c_size_t, False),
+                 "unsigned long long": (ctypes.c_ulonglong, False), "double": (ctypes.c_double, True)}
+    for name, params in decls.items():
+        ps = [] if params.strip() in ("", "void") else params.split(",")
+        argtypes = getattr(L, name).argtypes
+        assert argtypes is not None and len(argtypes) == len(ps), name
+        for p, t in zip(ps, argtypes):  # pointer-ness, then width and int / float class of scalars
+            is_ptr = t in (ctypes.c_void_p, ctypes.c_char_p) or issubclass(t, ctypes._Pointer)
+            assert ("*" in p) == is_ptr, (name, p)
+            if not is_ptr:
+                want, is_float = c_scalars[" ".join(p.split()[:-1]).replace("const ", "")]
+                assert ctypes.sizeof(t) == ctypes.sizeof(want), (name, p)
+                assert issubclass(t, (ctypes.c_double, ctypes.c_float)) == is_float, (name, p)
+
+
 def test_status_strings():
     L = aq.lib()
     for code in range(0, -8, -1):
