@@ -56,6 +56,28 @@ def test_binding_argument_counts_match_the_header():
                 assert issubclass(t, (ctypes.c_double, ctypes.c_float)) == is_float, (name, p)
 
 
+def test_packed_struct_layout_matches_the_header():
+    """AqPackedStruct lists aq_packed's fields in the header's order, with the
+    same widths (int32 scalars, pointers)."""
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "aq.h")).read(), flags=re.S)
+    body = re.search(r"typedef struct aq_packed \{(.*?)\} aq_packed;", src, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        ctype, names = decl.split(None, 1)
+        ptr = ctype.endswith("*") or names.startswith("*")
+        for n in names.replace("*", "").split(","):
+            fields.append((n.strip(), ptr, ctype.rstrip("*")))
+    py = aq.AqPackedStruct._fields_
+    assert [f[0] for f in fields] == [n for n, _ in py]
+    for (name, ptr, ctype), (_, t) in zip(fields, py):
+        assert (t is ctypes.c_void_p) == ptr, name
+        if not ptr:
+            assert ctype == "int32_t" and t is ctypes.c_int32, name
+
+
 def test_status_strings():
     L = aq.lib()
     for code in range(0, -8, -1):
