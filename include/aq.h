@@ -81,8 +81,9 @@ typedef enum { AQ_PHASE_DECODE = 0, AQ_PHASE_PREFILL = 1 } aq_phase;
  *
  * Inside a tile both precisions use the same element order: output row, then
  * input column.  w4, w8 and scales must start on a 16-byte boundary (the
- * kernels move them with bulk copies); a packed layout that breaks this is
- * rejected with AQ_ERR_ARG.
+ * kernels move them with bulk copies; fp32 tile scales need only 4 bytes) and
+ * tile_idx on a 4-byte one; a packed layout that breaks this is rejected with
+ * AQ_ERR_ARG.
  */
 typedef enum { AQ_SCALES_ROW_FP16 = 0, AQ_SCALES_TILE_FP32 = 1 } aq_scale_kind;
 
@@ -143,14 +144,16 @@ int aq_pack_metadata(const uint8_t* map_host, int R, int C, uint8_t* bitmap, int
 
 /*
  * Pack integer codes into the tile format (App. E.1, E.2; eq. 16, 17).
- *  codes  int8  [N][K] device, row-major: INT8 tiles any value, INT4 tiles in [-8, 7]
- *  scales fp16  [N][C] device (bits as uint16), sw[n][j]
+ *  codes  int8  [N][K] device, row-major, 16-byte aligned: INT8 tiles any value, INT4 tiles in [-8, 7]
+ *  scales fp16  [N][C] device (bits as uint16), 2-byte aligned, sw[n][j]
  *  map    uint8 [R][C] device, 1 = INT4 tile, 0 = INT8 tile
  *  out    host struct whose seven pointers the caller set to device buffers of
  *         aq_packed_sizes(N, K, bN, bK, out->T4) bytes; out->T4 must equal the
- *         number of INT4 labels in map.  The remaining fields are filled in.
+ *         number of INT4 labels in map; the buffers aligned as the struct's
+ *         description states.  The remaining fields are filled in.
  * Offline step: synchronizes `stream` and allocates a few bytes of temporary
- * device memory.  Errors: AQ_ERR_ARG (also when out->T4 disagrees with map),
+ * device memory.  Errors: AQ_ERR_ARG (also when out->T4 disagrees with map, or
+ * a pointer is misaligned),
  * AQ_ERR_SHAPE, AQ_ERR_RANGE (an INT4 tile holds a code outside [-8, 7]; the
  * output buffers are then unspecified), AQ_ERR_CUDA.
  */
@@ -187,7 +190,7 @@ int aq_pack_tiles(const int8_t* codes, const float* tile_scales, const uint8_t* 
  *         ldw >= K, ldw % 4 == 0 (fp32) or ldw % 8 == 0 (bf16); read only
  *  map    uint8 [R][C] device, 1 = INT4 tile, 0 = INT8 tile
  *  codes  int8  [N][K] device, 16-byte aligned (written)
- *  scales fp16  [N][C] device, bits as uint16 (written)
+ *  scales fp16  [N][C] device, bits as uint16, 2-byte aligned (written)
  * Offline step: synchronizes `stream` and allocates a few bytes of temporary
  * device memory.  Errors: AQ_ERR_ARG (null or misaligned pointer, bad wdtype
  * or search, ldw out of range, a label other than 0 or 1), AQ_ERR_SHAPE,
@@ -204,7 +207,7 @@ int aq_quantize_weights(const void* w, int wdtype, int N, int K, int ldw, int bN
  *   sx[m] = (float)s          (codes use the fp64 s; rint rounds half to even)
  *  x   bf16 [M][ldx] device (bits as uint16), 16-byte aligned, ldx % 8 == 0, ldx >= K
  *  xq  int8 [M][K] device, 16-byte aligned
- *  sx  fp32 [M] device
+ *  sx  fp32 [M] device, 4-byte aligned
  * 1 <= M, 16 <= K <= 1048576 with K % 16 == 0.  Errors: AQ_ERR_ARG, AQ_ERR_CUDA.
  */
 int aq_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream);
@@ -246,7 +249,7 @@ int aq_linear_prefill_expanded(const aq_packed* w, const int8_t* xq, const float
  *   xq = clamp(rint(x / s), -128, 127) (fp64 quotient)            sx = (float)s
  *  x   bf16 [M][ldx] device (bits as uint16), 16-byte aligned, ldx % 8 == 0, ldx >= K
  *  xq  int8 [M'][K] device, 8-byte aligned; padding rows receive zero codes
- *  sx  fp32 [M' / b_M][K / 64] device, row-major
+ *  sx  fp32 [M' / b_M][K / 64] device, row-major, 4-byte aligned
  * 1 <= M, 64 <= K <= 1048576 with K % 64 == 0.  Asynchronous on `stream`.
  * Errors: AQ_ERR_ARG, AQ_ERR_CUDA.  aq_act_group_rows: host only, b_M (0 for M < 1).
  */

@@ -193,6 +193,18 @@ def test_host_validation_rejects_before_any_launch():
     assert qw(16, 1, 128, 128, 132, 128, 128, 16, 1, 16, 16, None) == -1
     assert qw(20, 0, 128, 128, 128, 128, 128, 16, 1, 16, 16, None) == -1
     assert qw(16, 0, 128, 128, 128, 128, 128, 16, 1, 24, 16, None) == -1
+    assert qw(16, 0, 128, 128, 128, 128, 128, 16, 1, 16, 17, None) == -1   # fp16 scales are 2-byte words
+    # scalar words: activation scales (4 B), the tile table (4 B), fp16 row scales into the packer (2 B)
+    assert L.aq_quant_act(16, 1, 128, 128, 16, 18, None) == -1
+    assert L.aq_quant_act_groups(16, 1, 128, 128, 16, 18, None) == -1
+    odd_idx = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,
+                                bitmap=16, row_off4=16, row_off8=16, tile_idx=18, w4=16, w8=16, scales=16)
+    assert L.aq_linear_decode(ctypes.byref(odd_idx), 16, 16, 1, None, 16, 0, 128, 16, 1 << 20, None) == -1
+    assert L.aq_workspace_bytes(0, 1, ctypes.byref(odd_idx)) == 0
+    pk_out = aq.AqPackedStruct(T4=0, bitmap=16, row_off4=16, row_off8=16, tile_idx=18, w4=16, w8=16, scales=16)
+    assert L.aq_pack(16, 16, 16, 128, 128, 128, 128, ctypes.byref(pk_out), None) == -1
+    pk_out.tile_idx = 16
+    assert L.aq_pack(16, 17, 16, 128, 128, 128, 128, ctypes.byref(pk_out), None) == -1
     assert L.aq_workspace_bytes(0, 65, ctypes.byref(s)) == 0
     assert L.aq_workspace_bytes(0, 1, ctypes.byref(s)) >= 256
     assert L.aq_workspace_bytes(5, 1, ctypes.byref(s)) == 0
@@ -331,6 +343,11 @@ def test_paper_exact_mode_validation():
     assert lin(ctypes.byref(paper), 16, 16, 1, None, 18, 16, 128, None) == -1        # bias
     assert lin(ctypes.byref(paper), 16, 16, 1, None, None, 18, 128, None) == -1      # y
     assert L.aq_debug_paper_partials(ctypes.byref(paper), 16, 1, None, None) == -1
+    paper_odd_idx = aq.AqPackedStruct(N=128, K=128, bN=64, bK=64, R=2, C=2, T4=0, T8=4,
+                                      scale_kind=aq.AQ_SCALES_TILE_FP32, **dict(bufs, tile_idx=18))
+    assert lin(ctypes.byref(paper_odd_idx), 16, 16, 1, None, None, 16, 128, None) == -1
+    paper_out = aq.AqPackedStruct(T4=0, **bufs)
+    assert L.aq_pack_tiles(16, 18, 16, 128, 128, 64, 64, ctypes.byref(paper_out), None) == -1  # fp32 tile scales
     assert L.aq_debug_paper_partials(ctypes.byref(paper), 16, 1, 18, None) == -1    # P not 4-byte aligned
     # the per-token layer refuses a paper-form struct
     paper128 = aq.AqPackedStruct(N=128, K=128, bN=128, bK=128, R=1, C=1, T4=0, T8=1,

@@ -66,6 +66,7 @@ int validate_packed(const aq_packed* w) {
   if (!w->bitmap || !w->row_off4 || !w->row_off8 || !w->tile_idx || !w->scales) return AQ_ERR_ARG;
   if ((w->T4 > 0 && !w->w4) || (w->T8 > 0 && !w->w8)) return AQ_ERR_ARG;
   if (((uintptr_t)w->w4 & 15) || ((uintptr_t)w->w8 & 15) || ((uintptr_t)w->scales & 15)) return AQ_ERR_ARG;
+  if ((uintptr_t)w->tile_idx & 3) return AQ_ERR_ARG;  // read as 4-byte words
   return AQ_OK;
 }
 
@@ -182,7 +183,7 @@ extern "C" size_t aq_workspace_bytes(int phase, int M, const aq_packed* w) {
 
 extern "C" int aq_quant_act(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream) {
   if (!x || !xq || !sx || M < 1 || K < 16 || K % 16 || K > (1 << 20) || ldx < K || ldx % 8) return AQ_ERR_ARG;
-  if (((uintptr_t)x & 15) || ((uintptr_t)xq & 15)) return AQ_ERR_ARG;
+  if (((uintptr_t)x & 15) || ((uintptr_t)xq & 15) || ((uintptr_t)sx & 3)) return AQ_ERR_ARG;
   return launch_quant_act(x, M, K, ldx, xq, sx, static_cast<cudaStream_t>(stream)) == cudaSuccess ? AQ_OK
                                                                                                    : AQ_ERR_CUDA;
 }
@@ -248,7 +249,7 @@ extern "C" int aq_act_group_rows(int M) { return M < 1 ? 0 : act_group_rows(M); 
 
 extern "C" int aq_quant_act_groups(const uint16_t* x, int M, int K, int ldx, int8_t* xq, float* sx, void* stream) {
   if (!x || !xq || !sx || M < 1 || K < 64 || K % 64 || K > (1 << 20) || ldx < K || ldx % 8) return AQ_ERR_ARG;
-  if (((uintptr_t)x & 15) || ((uintptr_t)xq & 7)) return AQ_ERR_ARG;
+  if (((uintptr_t)x & 15) || ((uintptr_t)xq & 7) || ((uintptr_t)sx & 3)) return AQ_ERR_ARG;
   return launch_quant_act_groups(x, M, K, ldx, xq, sx, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? AQ_OK : AQ_ERR_CUDA;
 }

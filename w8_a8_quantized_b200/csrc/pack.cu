@@ -128,6 +128,10 @@ static int pack_common(const int8_t* codes, const uint16_t* scales, const float*
   if (!out->bitmap || !out->row_off4 || !out->row_off8 || !out->tile_idx || !out->scales) return AQ_ERR_ARG;
   if ((out->T4 > 0 && !out->w4) || (out->T4 < T && !out->w8)) return AQ_ERR_ARG;
   if (tile_scales != nullptr && ((uintptr_t)out->scales & 3)) return AQ_ERR_ARG;
+  // scalar words: tile table (4 B), fp16 row scales (2 B), fp32 tile scales (4 B)
+  if (((uintptr_t)out->tile_idx & 3) || ((uintptr_t)out->scales & 1) || ((uintptr_t)scales & 1) ||
+      ((uintptr_t)tile_scales & 3))
+    return AQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   std::vector<uint8_t> map_h(T), bitmap_h((T + 7) / 8);

@@ -250,6 +250,7 @@ int validate_paper_packed(const aq_packed* w) {
   if (!w->bitmap || !w->tile_idx || !w->scales) return AQ_ERR_ARG;
   if ((w->T4 > 0 && !w->w4) || (w->T8 > 0 && !w->w8)) return AQ_ERR_ARG;
   if (((uintptr_t)w->w4 & 15) || ((uintptr_t)w->w8 & 15) || ((uintptr_t)w->scales & 3)) return AQ_ERR_ARG;
+  if ((uintptr_t)w->tile_idx & 3) return AQ_ERR_ARG;
   return AQ_OK;
 }
 

@@ -197,6 +197,7 @@ extern "C" int aq_quantize_weights(const void* w, int wdtype, int N, int K, int 
                                    const uint8_t* map, int search, int8_t* codes, uint16_t* scales, void* stream) {
   using namespace aq;
   if (!w || !map || !codes || !scales) return AQ_ERR_ARG;
+  if ((uintptr_t)scales & 1) return AQ_ERR_ARG;  // fp16 scales written as 2-byte words
   if (wdtype != AQ_F32 && wdtype != AQ_BF16) return AQ_ERR_ARG;
   if (search != 0 && search != 1) return AQ_ERR_ARG;
   if (!geometry_ok(N, K, bN, bK)) return AQ_ERR_SHAPE;
