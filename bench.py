@@ -752,9 +752,11 @@ def run_reference(args, wl, peaks):
     decode = wl["phase"] == "decode"
     unit = "GB/s" if decode else "TOPS"
     value = tot_b / tot_t / 1e9 if decode else 2.0 * tot_macs / tot_t / 1e12
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     desc = (f"one whole projection of layer 0 per step (cycling through the layer's projections), "
-            f"{rows} token(s): unpack + quantize + tile products + fp64 rescale")
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+            f"{rows} token(s): unpack + quantize + tile products + fp64 rescale"
+            + (f"; rank 0 of {world} alone" if world > 1 else ""))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": tot_t / max(args.steps, 1) * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "model_shape": wl["model"], "phase": wl["phase"],

@@ -68,3 +68,24 @@ def test_cpu_baseline_reports_rate_and_measured_cores():
     assert 1.0 <= out["cores"] <= (os.cpu_count() or 1) + 0.5
     short = bench.cpu_baseline(wl, 0.05, True, legs=("all_cores",))
     assert "single_thread" not in short and short["value"] > 0
+
+
+def test_reference_arm_prints_one_line_from_rank_zero():
+    """`bench.py --impl reference` under a 2-rank launch: rank 0 times the oracle
+    and prints the one JSON line, the other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "2", "--warmup", "1"]
+    out = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=240)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
